@@ -1,0 +1,318 @@
+/*
+ * lq_oracle.c -- plain, slow, fp64 CPU oracle for the LiftQuant decode operator.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the smoke check and the benchmark's
+ * CPU-baseline leg may build, load or call this file. The library under
+ * fractional_bit_weight_b200/ never does, and shares no code, header, table or
+ * constant with it.
+ *
+ * What it computes (sources are the pages on LiftQuant):
+ *   - "LiftQuant: Continuous Bit-Width LLM Quantization via Dimensional Lifting
+ *     and Projection" (paper translation, bittide.aicompass.dev), sec. 3.1:
+ *     every length-d weight block is w ~= M * w_q with w_q in {+1,-1}^D and
+ *     w_i = sum_j M_ij (w_q)_j; M is the d x D mapping matrix.
+ *   - same paper, sec. 3 (intro) and sec. 2: the bit-width is D/d and the
+ *     fused decode operator is o = diag(s) W (M T a).
+ *   - "Paper Review: LiftQuant" (romaanj.github.io), "Method": decode is
+ *     diag(s) * W_q * (T* a) with T* the lift fused with the whitening T,
+ *     and T is Hadamard-initialised orthogonal mixing plus scalings.
+ *
+ * Readings taken where the pages are silent (each is listed in the design notes):
+ *   - T acts on contiguous blocks of Bh inputs: xt = H_Bh (sigma . c . x) / sqrt(Bh),
+ *     H in Sylvester (natural) order, H[i][j] = (-1)^popcount(i & j);
+ *     Bh = 0 means T is the identity.
+ *   - K is zero-padded up to G*d (G = ceil(K/d)) after T.
+ *   - Bitstream LQ_FORMAT_V1: row n, block g, lifted coordinate j is bit
+ *     q = g*D + j of the row; bit q lives in byte q/8 at bit position q%8
+ *     (LSB first); a set bit means w_q = -1; each row is zero-padded to a
+ *     multiple of 16 bytes.
+ *
+ * Everything below is written as the plain definition: explicit dense H, an
+ * explicit weight row W[n][.] = blockwise M * b, and an fp64 dot product.
+ * Threads (OpenMP) split output rows only; each row is computed by one thread
+ * in a fixed order, so results do not depend on the thread count.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ---------------------------------------------------------------- sizes */
+
+/* Number of length-d blocks in a row of K inputs (K zero-padded to G*d). */
+static int64_t orc_groups(int32_t K, int32_t d) { return ((int64_t)K + d - 1) / d; }
+
+static int orc_valid_code(int32_t K, int32_t d, int32_t D) {
+  return K >= 1 && d >= 1 && D >= d && D <= 32;
+}
+
+/* Lifted length of a row = number of stored bits = G*D. */
+int64_t orc_lifted_bits(int32_t K, int32_t d, int32_t D) {
+  if (!orc_valid_code(K, d, D)) return -1;
+  return orc_groups(K, d) * D;
+}
+
+/* Bytes per stored row: ceil(G*D / 8) rounded up to a multiple of 16. */
+int64_t orc_row_bytes(int32_t K, int32_t d, int32_t D) {
+  int64_t bits = orc_lifted_bits(K, d, D);
+  if (bits < 0) return -1;
+  int64_t bytes = (bits + 7) / 8;
+  return (bytes + 15) / 16 * 16;
+}
+
+/* ---------------------------------------------------------------- packing */
+
+/* b: [N][G*D] int8 entries in {+1,-1}; out: [N][row_bytes] bytes.
+ * Returns 0, or -1 if an entry of b is not +1/-1 or the sizes are invalid. */
+int orc_pack(const int8_t* b, int64_t N, int32_t K, int32_t d, int32_t D, uint8_t* out) {
+  int64_t bits = orc_lifted_bits(K, d, D);
+  int64_t rb = orc_row_bytes(K, d, D);
+  if (bits < 0 || N < 0) return -1;
+  memset(out, 0, (size_t)(N * rb));
+  for (int64_t n = 0; n < N; ++n) {
+    const int8_t* br = b + n * bits;
+    uint8_t* orow = out + n * rb;
+    for (int64_t q = 0; q < bits; ++q) {
+      if (br[q] == -1) {
+        orow[q / 8] |= (uint8_t)(1u << (q % 8));
+      } else if (br[q] != 1) {
+        return -1;
+      }
+    }
+  }
+  return 0;
+}
+
+/* Inverse of orc_pack. Padding bits are ignored. */
+int orc_unpack(const uint8_t* packed, int64_t N, int32_t K, int32_t d, int32_t D, int8_t* b) {
+  int64_t bits = orc_lifted_bits(K, d, D);
+  int64_t rb = orc_row_bytes(K, d, D);
+  if (bits < 0 || N < 0) return -1;
+  for (int64_t n = 0; n < N; ++n) {
+    const uint8_t* prow = packed + n * rb;
+    for (int64_t q = 0; q < bits; ++q) {
+      int bit = (prow[q / 8] >> (q % 8)) & 1;
+      b[n * bits + q] = bit ? (int8_t)-1 : (int8_t)1;
+    }
+  }
+  return 0;
+}
+
+/* ---------------------------------------------------------------- whitening */
+
+static int orc_parity(uint32_t v) {
+  int p = 0;
+  while (v) {
+    p ^= (int)(v & 1u);
+    v >>= 1;
+  }
+  return p;
+}
+
+/* Entry (i, j) of the Sylvester-ordered Hadamard matrix. */
+static double orc_hadamard_entry(int32_t i, int32_t j) {
+  return orc_parity((uint32_t)(i & j)) ? -1.0 : 1.0;
+}
+
+static int orc_is_pow2(int32_t v) { return v > 0 && (v & (v - 1)) == 0; }
+
+/* xt[t][k] = T(x[t])[k] for batch rows of K inputs.
+ * sign: [K] entries +1/-1 or NULL (all +1); chan_scale: [K] or NULL (all 1).
+ * block = 0: T is the identity (sign and chan_scale unused).
+ * Returns 0, or -1 on invalid sizes. Dense O(K * block) per row, on purpose. */
+int orc_whiten(const double* x, int64_t batch, int32_t K, const int8_t* sign,
+               const double* chan_scale, int32_t block, double* xt) {
+  if (K < 1 || batch < 0) return -1;
+  if (block == 0) {
+    memcpy(xt, x, (size_t)(batch * K) * sizeof(double));
+    return 0;
+  }
+  if (!orc_is_pow2(block) || K % block != 0) return -1;
+  const double norm = 1.0 / sqrt((double)block);
+  double* u = (double*)malloc((size_t)block * sizeof(double));
+  if (!u) return -1;
+  for (int64_t t = 0; t < batch; ++t) {
+    const double* xr = x + t * K;
+    double* yr = xt + t * K;
+    for (int32_t b0 = 0; b0 < K; b0 += block) {
+      for (int32_t j = 0; j < block; ++j) {
+        double v = xr[b0 + j];
+        if (chan_scale) v *= chan_scale[b0 + j];
+        if (sign) v *= (double)sign[b0 + j];
+        u[j] = v;
+      }
+      for (int32_t i = 0; i < block; ++i) {
+        double acc = 0.0;
+        for (int32_t j = 0; j < block; ++j) acc += orc_hadamard_entry(i, j) * u[j];
+        yr[b0 + i] = acc * norm;
+      }
+    }
+  }
+  free(u);
+  return 0;
+}
+
+/* ---------------------------------------------------------------- lift */
+
+/* z[t][g*D + j] = sum_i M[i][j] * xt[t][g*d + i], with xt zero beyond K.
+ * This is the lifted activation (M^T applied per block), computed after T.
+ * M: [d][D] row-major. z: [batch][G*D]. */
+int orc_lift(const double* x, int64_t batch, int32_t K, const int8_t* sign,
+             const double* chan_scale, int32_t block, const double* M, int32_t d, int32_t D,
+             double* z) {
+  if (!orc_valid_code(K, d, D) || batch < 0) return -1;
+  const int64_t G = orc_groups(K, d);
+  double* xt = (double*)malloc((size_t)(batch * K) * sizeof(double));
+  if (!xt) return -1;
+  if (orc_whiten(x, batch, K, sign, chan_scale, block, xt) != 0) {
+    free(xt);
+    return -1;
+  }
+  for (int64_t t = 0; t < batch; ++t) {
+    for (int64_t g = 0; g < G; ++g) {
+      for (int32_t j = 0; j < D; ++j) {
+        double acc = 0.0;
+        for (int32_t i = 0; i < d; ++i) {
+          int64_t k = g * d + i;
+          double v = (k < K) ? xt[t * K + k] : 0.0;
+          acc += M[i * D + j] * v;
+        }
+        z[t * G * D + g * D + j] = acc;
+      }
+    }
+  }
+  free(xt);
+  return 0;
+}
+
+/* ---------------------------------------------------------------- forward */
+
+/* y[t][n] = s[n] * sum_{k<K} W[n][k] * T(x[t])[k], with W[n][g*d+i] = sum_j M[i][j] b[n][g][j]
+ * and b unpacked from the LQ_FORMAT_V1 rows in `packed` ([nrows][row_bytes]).
+ * s: [nrows]. y: [batch][nrows]. nthreads <= 0 means one thread.
+ * This forms each weight row explicitly, the plain definition of the operator. */
+int orc_forward(const double* x, int64_t batch, int32_t K, int64_t nrows, int32_t d, int32_t D,
+                const uint8_t* packed, const double* M, const double* s, const int8_t* sign,
+                const double* chan_scale, int32_t block, double* y, int nthreads) {
+  if (!orc_valid_code(K, d, D) || batch < 0 || nrows < 0) return -1;
+  const int64_t G = orc_groups(K, d);
+  const int64_t bits = G * D;
+  const int64_t rb = orc_row_bytes(K, d, D);
+  double* xt = (double*)malloc((size_t)(batch * K + 1) * sizeof(double));
+  if (!xt) return -1;
+  if (orc_whiten(x, batch, K, sign, chan_scale, block, xt) != 0) {
+    free(xt);
+    return -1;
+  }
+  int failed = 0;
+  if (nthreads < 1) nthreads = 1;
+#pragma omp parallel num_threads(nthreads)
+  {
+    int8_t* br = (int8_t*)malloc((size_t)bits);
+    double* w = (double*)malloc((size_t)(G * d) * sizeof(double));
+    if (!br || !w) {
+#pragma omp atomic write
+      failed = 1;
+    }
+#pragma omp for schedule(static)
+    for (int64_t n = 0; n < nrows; ++n) {
+      if (!br || !w) continue;
+      orc_unpack(packed + n * rb, 1, K, d, D, br);
+      for (int64_t g = 0; g < G; ++g) {
+        for (int32_t i = 0; i < d; ++i) {
+          double acc = 0.0;
+          for (int32_t j = 0; j < D; ++j) acc += M[i * D + j] * (double)br[g * D + j];
+          w[g * d + i] = acc;
+        }
+      }
+      for (int64_t t = 0; t < batch; ++t) {
+        double acc = 0.0;
+        for (int32_t k = 0; k < K; ++k) acc += w[k] * xt[t * K + k];
+        y[t * nrows + n] = s[n] * acc;
+      }
+    }
+    free(br);
+    free(w);
+  }
+  free(xt);
+  return failed ? -1 : 0;
+}
+
+/* Same operator in the lifted form: y[t][n] = s[n] * sum_q b[n][q] * z[t][q], with z from
+ * orc_lift. Used to check the identity b^T (M^T x) = (M b)^T x against orc_forward. */
+int orc_forward_lifted(const double* x, int64_t batch, int32_t K, int64_t nrows, int32_t d,
+                       int32_t D, const uint8_t* packed, const double* M, const double* s,
+                       const int8_t* sign, const double* chan_scale, int32_t block, double* y,
+                       int nthreads) {
+  if (!orc_valid_code(K, d, D) || batch < 0 || nrows < 0) return -1;
+  const int64_t bits = orc_lifted_bits(K, d, D);
+  const int64_t rb = orc_row_bytes(K, d, D);
+  double* z = (double*)malloc((size_t)(batch * bits + 1) * sizeof(double));
+  if (!z) return -1;
+  if (orc_lift(x, batch, K, sign, chan_scale, block, M, d, D, z) != 0) {
+    free(z);
+    return -1;
+  }
+  int failed = 0;
+  if (nthreads < 1) nthreads = 1;
+#pragma omp parallel num_threads(nthreads)
+  {
+    int8_t* br = (int8_t*)malloc((size_t)bits);
+    if (!br) {
+#pragma omp atomic write
+      failed = 1;
+    }
+#pragma omp for schedule(static)
+    for (int64_t n = 0; n < nrows; ++n) {
+      if (!br) continue;
+      orc_unpack(packed + n * rb, 1, K, d, D, br);
+      for (int64_t t = 0; t < batch; ++t) {
+        double acc = 0.0;
+        for (int64_t q = 0; q < bits; ++q) acc += (double)br[q] * z[t * bits + q];
+        y[t * nrows + n] = s[n] * acc;
+      }
+    }
+    free(br);
+  }
+  free(z);
+  return failed ? -1 : 0;
+}
+
+/* ---------------------------------------------------------------- encoder */
+
+/* Nearest codeword by exhaustive search, the inner minimisation of Eq. (1) of the paper:
+ * argmin over b in {+1,-1}^D of || w - M b ||^2, w in R^d.
+ * Codeword c has b_j = -1 exactly when bit j of c is set; ties keep the smallest c.
+ * b_out: [D]. Returns the codeword index c, or -1 if D > 24 or sizes are invalid. */
+int64_t orc_encode_bruteforce(const double* w, const double* M, int32_t d, int32_t D,
+                              int8_t* b_out) {
+  if (d < 1 || D < 1 || D > 24) return -1;
+  int64_t best = -1;
+  double best_dist = 0.0;
+  for (int64_t c = 0; c < ((int64_t)1 << D); ++c) {
+    double dist = 0.0;
+    for (int32_t i = 0; i < d; ++i) {
+      double r = w[i];
+      for (int32_t j = 0; j < D; ++j) r -= M[i * D + j] * (((c >> j) & 1) ? -1.0 : 1.0);
+      dist += r * r;
+    }
+    if (best < 0 || dist < best_dist) {
+      best = c;
+      best_dist = dist;
+    }
+  }
+  for (int32_t j = 0; j < D; ++j) b_out[j] = ((best >> j) & 1) ? (int8_t)-1 : (int8_t)1;
+  return best;
+}
+
+int orc_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
