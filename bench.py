@@ -1,0 +1,437 @@
+"""Benchmark of the LiftQuant decode operator (lq_gemm) on B200.
+
+One step = one lq_gemm call (whiten + lift + +-1 contraction + row scale) over one batch of
+synthetic inputs already resident in HBM. The default workload is the Llama-2-7B q_proj
+shape (K = N = 4096, d = 10, D = 24: 2.4 bit, batch 1, block-256 Hadamard whitening).
+Inputs rotate over enough copies of the packed weights that successive steps never hit in
+L2. Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl lq|reference]
+
+Multi-GPU: independent replicas (one process per GPU, launched by torchrun); the path has
+no exchange step, so the ranks only meet for the barrier and the max-over-ranks timing.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import fractional_bit_weight_b200 as lq  # noqa: E402
+from fractional_bit_weight_b200 import synth  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+# name -> (workload spec index into synth.workload_specs(cfg), cfg, metric kind)
+WORKLOADS = {
+    "llama2_7b_qproj_b1": (2, 0, "gemv"),
+    "llama3_70b_gateup_b1": (3, 0, "gemv"),
+    "llama3_70b_gateup_b16": (3, 2, "gemv"),
+    "llama3_70b_down_b1": (3, 3, "gemv"),
+    "sweep_d10D24_b1": (4, 8, "gemv"),
+    "prefill_b2048": (5, 0, "gemm"),
+}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", default="lq", choices=["lq", "reference"])
+    p.add_argument("--workload", default="llama2_7b_qproj_b1", choices=sorted(WORKLOADS))
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v, ws):
+    if ws == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def csrc_digest():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "fractional_bit_weight_b200", "csrc")
+    for name in sorted(os.listdir(d)):
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu summary, if it was
+    taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = rec.get(workload)
+    if not ent or ent.get("csrc_digest") != csrc_digest():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    def __init__(self, index):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _sample(self):
+        nv = self._nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+        r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        names = {
+            "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap,
+            "hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+            "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+            "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+            "hw_power_brake_slowdown": nv.nvmlClocksEventReasonHwPowerBrakeSlowdown,
+        }
+        for k, bit in names.items():
+            if r & bit:
+                self.reasons.add(k)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                return
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- workload on the device
+
+class DeviceWorkload:
+    def __init__(self, spec, dev):
+        name, seed, li, K, N, d, D, batch, kw = spec
+        self.name, self.K, self.N, self.d, self.D, self.batch = name, K, N, d, D, batch
+        layer = synth.build(spec, with_bits=False)     # sign, M, s, x from the seeded recipe
+        self.layer = layer
+        self.block = layer.block
+        self.L = lq.lifted_bits(K, d, D)
+        self.packed_bytes = N * self.L // 8 if self.L % 8 == 0 else N * self.L / 8
+        self.row_words = lq.row_stride_bytes(K, d, D) // 4
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed * 1000 + li)
+        # rotate over copies so that the bytes streamed between reuses exceed 3x L2
+        stored = N * self.row_words * 4
+        self.ncopies = max(1, min(64, math.ceil(3 * L2_BYTES / stored)))
+        self.packed = []
+        for _ in range(self.ncopies):
+            b = (torch.randint(0, 2, (N, self.L), generator=g, device=dev, dtype=torch.int8)
+                 * 2 - 1).to(torch.int8)
+            self.packed.append(lq.pack(b, K, d, D))
+            del b
+        self.x = _x_tensor(layer).to(dev)
+        self.s = torch.from_numpy(np.ascontiguousarray(layer.s_raw)).to(dev)
+        self.M = torch.from_numpy(layer.M).to(dev)
+        self.sign = torch.from_numpy(layer.sign).to(dev)
+        self.y = torch.empty((batch, N), dtype=torch.float32, device=dev)
+        self.ws = lq.new_workspace(batch, K, N, d, D, device=dev)
+        self.stored_bytes = stored
+
+    def step(self, i, x=None, y=None):
+        lq.gemm(self.x if x is None else x, self.packed[i % self.ncopies], self.M, self.s,
+                self.d, self.D, sign=self.sign, block=self.block,
+                y=self.y if y is None else y, workspace=self.ws)
+
+    def algorithmic_bytes(self):
+        """Bytes one call must move at minimum: packed codes, s, x, y, M, sign."""
+        return (self.packed_bytes + self.s.numel() * self.s.element_size()
+                + self.x.numel() * self.x.element_size() + self.y.numel() * 4
+                + self.M.numel() * 4 + self.sign.numel())
+
+    def flops(self):
+        """Contraction + lift + FWHT flops of one call (lifted form)."""
+        G = -(-self.K // self.d)
+        fwht = self.batch * self.K * int(math.log2(self.block)) if self.block else 0
+        return 2.0 * self.batch * self.N * self.L + 2.0 * self.batch * G * self.d * self.D + fwht
+
+
+def _x_tensor(layer):
+    if layer.x_dtype == synth.BF16:
+        return torch.from_numpy(layer.x_raw.view(np.int16).copy()).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(layer.x_raw))
+
+
+def kernels_per_step():
+    return 2      # lift prologue + contraction
+
+
+def time_steps(fn, steps, warmup, ws):
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        fn(warmup + i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / 1e3   # seconds
+
+
+# ---------------------------------------------------------------- CPU oracle baseline
+
+def cpu_oracle_run(wl, budget_s=10.0, max_rows=None):
+    """Times the fp64 oracle on the host cores over a bounded sample of rows of the same
+    workload; returns (value in the workload's unit, sample description, threads)."""
+    import oracle
+    threads = len(os.sched_getaffinity(0))
+    layer = wl.layer
+    rng = np.random.Generator(np.random.PCG64(0))
+    # measure one small batch of rows to size the sample, then run the sample
+    probe = min(wl.N, 64)
+    rows = np.arange(probe)
+    b = synth.random_signs(rng, (probe, wl.L))
+    p = oracle.pack(b, wl.K, wl.d, wl.D)
+    t0 = time.perf_counter()
+    oracle.forward(layer.x, p, layer.M, layer.s[rows], wl.d, wl.D, sign=layer.sign,
+                   block=layer.block, nthreads=threads)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    n = int(min(wl.N if max_rows is None else max_rows, max(probe, probe * budget_s / dt)))
+    b = synth.random_signs(rng, (n, wl.L))
+    p = oracle.pack(b, wl.K, wl.d, wl.D)
+    s = np.resize(layer.s, n)
+    t0 = time.perf_counter()
+    oracle.forward(layer.x, p, layer.M, s, wl.d, wl.D, sign=layer.sign, block=layer.block,
+                   nthreads=threads)
+    dt = time.perf_counter() - t0
+    frac = n / wl.N
+    sample = (f"{n} of {wl.N} rows x batch {wl.batch} ({frac:.3f} of one call), fp64 oracle, "
+              f"{threads} OpenMP threads")
+    return frac, dt, sample, threads
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    args = parse()
+    ws, rank, local = dist_setup()
+    cfg, idx, kind = WORKLOADS[args.workload]
+    spec = synth.workload_specs(cfg)[idx]
+    if args.impl == "reference":
+        return reference_arm(args, spec, kind, ws, rank)
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = DeviceWorkload(spec, dev)
+    peaks, peak_src = measured_peaks()
+
+    with ClockSampler(local) as clk:
+        secs = time_steps(wl.step, args.steps, args.warmup, ws)
+    secs = max_over_ranks(secs, ws)
+    per_step = secs / args.steps
+
+    total_packed = wl.packed_bytes * args.steps * ws
+    gbs = total_packed / secs / 1e9
+    tflops = wl.flops() * args.steps * ws / secs / 1e12
+    if kind == "gemv":
+        metric, value, unit = "lq_gemv_packed_weight_GBps", gbs, "GB/s"
+        achieved = wl.algorithmic_bytes() / per_step / 1e9
+        peak = float(peaks["hbm_gbs"])
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
+                "peak_source": f"{peak_src} hbm_gbs (copy, read+write)",
+                "packed_frac": wl.packed_bytes / per_step / 1e9 / peak}
+    else:
+        metric, value, unit = "lq_prefill_gemm_TFLOPs", tflops, "TFLOP/s"
+        achieved = wl.flops() / per_step / 1e12
+        peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
+                "peak_source": f"{peak_src} bf16_tflops_sustained (fp16 dense = bf16 dense)"}
+
+    out = {
+        "metric": metric, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded: random sign codes, N(0,1/D) M, N(0,1) bf16 x)",
+        "config": {"workload": wl.name, "K": wl.K, "N": wl.N, "d": wl.d, "D": wl.D,
+                   "batch": wl.batch, "bits_per_weight": wl.D / wl.d, "hadamard_block": wl.block,
+                   "packed_bytes": wl.packed_bytes, "parallelism": f"replicas x{ws}",
+                   "l2": f"rotating {wl.ncopies} copies of the packed weights "
+                         f"({wl.ncopies * wl.stored_bytes / 1e6:.0f} MB > L2)"},
+        "roofline": roof,
+        "gpu_launches": kernels_per_step() * args.steps,
+        "clocks": clk.summary(),
+    }
+    if kind == "gemv":
+        out["tflops"] = tflops
+    if not args.no_e2e:
+        out["e2e"] = e2e_run(wl, args, ws)
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        frac, dt, sample, threads = cpu_oracle_run(wl)
+        cpu_val = (wl.packed_bytes * frac / dt / 1e9) if kind == "gemv" else \
+            (wl.flops() * frac / dt / 1e12)
+        out["cpu_baseline"] = {"value": cpu_val, "unit": unit, "cores": threads, "kind": "oracle",
+                               "sample": sample}
+    if rank == 0:
+        print(json.dumps(out))
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+def e2e_run(wl, args, ws):
+    """Same metric through the public call with host buffers: every step copies x from pinned
+    host memory to the device and y back, inside the timed region."""
+    x_host = wl.x.cpu().pin_memory()
+    y_host = torch.empty(wl.y.shape, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(wl.x)
+
+    def step(i):
+        x_dev.copy_(x_host, non_blocking=True)
+        wl.step(i, x=x_dev)
+        y_host.copy_(wl.y, non_blocking=True)
+
+    secs = max_over_ranks(time_steps(step, args.steps, args.warmup, ws), ws)
+    if wl.flops() and WORKLOADS[args.workload][2] == "gemm":
+        v, u = wl.flops() * args.steps * ws / secs / 1e12, "TFLOP/s"
+    else:
+        v, u = wl.packed_bytes * args.steps * ws / secs / 1e9, "GB/s"
+    return {"value": v, "unit": u, "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+            "d2h_bytes_per_step": y_host.numel() * 4}
+
+
+def reference_arm(args, spec, kind, ws, rank):
+    """The oracle, as it stands, on the host cores: each step is a bounded sample of the
+    workload. Under torchrun only rank 0 runs it."""
+    if rank != 0:
+        if ws > 1:
+            torch.distributed.destroy_process_group()
+        return
+    import oracle
+    name, seed, li, K, N, d, D, batch, kw = spec
+    layer = synth.build(spec, with_bits=False)
+    L = lq_free_lifted_bits(K, d, D)
+    threads = len(os.sched_getaffinity(0))
+    rng = np.random.Generator(np.random.PCG64(1))
+    rows = min(N, 256 if kind == "gemv" else 16)
+    toks = min(batch, 64)
+    b = synth.random_signs(rng, (rows, L))
+    p = oracle.pack(b, K, d, D)
+    x = layer.x[:toks]
+
+    def step():
+        oracle.forward(x, p, layer.M, layer.s[:rows], d, D, sign=layer.sign, block=layer.block,
+                       nthreads=threads)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    secs = time.perf_counter() - t0
+    frac = rows / N * toks / batch
+    packed = N * L / 8
+    G = -(-K // d)
+    flops = 2.0 * batch * N * L + 2.0 * batch * G * d * D
+    if kind == "gemv":
+        metric, unit = "lq_gemv_packed_weight_GBps", "GB/s"
+        value = packed * frac * args.steps / secs / 1e9
+    else:
+        metric, unit = "lq_prefill_gemm_TFLOPs", "TFLOP/s"
+        value = flops * frac * args.steps / secs / 1e12
+    sample = f"{rows} of {N} rows x {toks} of {batch} tokens per step, fp64 oracle"
+    out = {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": ws,
+           "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": name, "K": K, "N": N, "d": d, "D": D, "batch": batch},
+           "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out))
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+def lq_free_lifted_bits(K, d, D):
+    return (K + d - 1) // d * D
+
+
+if __name__ == "__main__":
+    main()

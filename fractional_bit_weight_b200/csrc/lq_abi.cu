@@ -1,0 +1,250 @@
+// lq_abi.cu -- the extern "C" entry points of liblq: argument checks, planning, launches.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "lq_internal.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+lq_status fail(lq_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+lq_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(LQ_ECUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+void clear_error() { g_last_error[0] = '\0'; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool valid_code(int32_t K, int32_t d, int32_t D) {
+  return K >= 1 && d >= 1 && D >= d && D <= LQ_MAX_D;
+}
+
+int64_t lifted_bits(int32_t K, int32_t d, int32_t D) {
+  return ((int64_t)K + d - 1) / d * D;
+}
+
+int64_t row_stride_bytes(int32_t K, int32_t d, int32_t D) {
+  const int64_t bytes = (lifted_bits(K, d, D) + 7) / 8;
+  return (bytes + 15) / 16 * 16;
+}
+
+bool valid_dtype(lq_dtype t) { return t == LQ_F32 || t == LQ_F16 || t == LQ_BF16; }
+
+size_t dtype_size(lq_dtype t) { return t == LQ_F32 ? 4 : 2; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Validates a whitening descriptor against K and converts it.
+lq_status make_whiten(const lq_whiten_desc* T, int32_t K, lq::Whiten* out) {
+  out->sign = nullptr;
+  out->chan_scale = nullptr;
+  out->block = 0;
+  out->inv_sqrt = 1.f;
+  if (T == nullptr || T->block == 0) return LQ_OK;
+  const int32_t B = T->block;
+  if (B < 0 || (B & (B - 1)) != 0)
+    return fail(LQ_EINVAL, "whitening block %d is not 0 or a power of two", B);
+  if (B > LQ_MAX_HADAMARD)
+    return fail(LQ_EUNSUPPORTED, "whitening block %d exceeds LQ_MAX_HADAMARD (%d)", B,
+                LQ_MAX_HADAMARD);
+  if (K % B != 0) return fail(LQ_EINVAL, "whitening block %d does not divide K = %d", B, K);
+  out->sign = T->sign;
+  out->chan_scale = T->chan_scale;
+  out->block = B;
+  out->inv_sqrt = (float)(1.0 / std::sqrt((double)B));
+  if (out->chan_scale && !aligned(out->chan_scale, 4))
+    return fail(LQ_EINVAL, "chan_scale is not 4-byte aligned");
+  return LQ_OK;
+}
+
+// Workspace layout of lq_gemm (byte offsets, all 256-aligned).
+struct WsLayout {
+  size_t counters;   // uint32 [ntg * ntiles]
+  size_t z;          // float  [batch][L]
+  size_t partials;   // float  [nsl][batch][N]
+  size_t total;
+  lq::GemvPlan gemv;
+};
+
+WsLayout layout_gemm(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D) {
+  WsLayout w{};
+  const int64_t L = lifted_bits(K, d, D);
+  w.gemv = lq::plan_gemv(batch, L, N);
+  size_t off = sizeof(lq::WsHeader);
+  w.counters = off;
+  off = round_up(off + (size_t)w.gemv.ntg * w.gemv.ntiles * sizeof(uint32_t), 256);
+  w.z = off;
+  off = round_up(off + (size_t)batch * L * sizeof(float), 256);
+  w.partials = off;
+  if (w.gemv.nsl > 1) off = round_up(off + (size_t)w.gemv.nsl * batch * N * sizeof(float), 256);
+  w.total = off;
+  return w;
+}
+
+constexpr int32_t kMaxBatch = 1 << 20;
+constexpr int32_t kMaxK = 1 << 24;
+
+}  // namespace
+
+extern "C" {
+
+int32_t lq_abi_version(void) { return LQ_ABI_VERSION; }
+
+int64_t lq_lifted_bits(int32_t K, int32_t d, int32_t D) {
+  return valid_code(K, d, D) ? lifted_bits(K, d, D) : -1;
+}
+
+int64_t lq_row_stride_bytes(int32_t K, int32_t d, int32_t D) {
+  return valid_code(K, d, D) ? row_stride_bytes(K, d, D) : -1;
+}
+
+const char* lq_status_string(lq_status s) {
+  switch (s) {
+    case LQ_OK: return "LQ_OK";
+    case LQ_EINVAL: return "LQ_EINVAL: invalid argument";
+    case LQ_EUNSUPPORTED: return "LQ_EUNSUPPORTED: valid but not supported";
+    case LQ_ECUDA: return "LQ_ECUDA: CUDA error";
+    case LQ_ETIMEOUT: return "LQ_ETIMEOUT: device-side wait expired";
+    case LQ_EDEVICE: return "LQ_EDEVICE: device-side check failed";
+  }
+  return "unknown lq_status";
+}
+
+const char* lq_last_error(void) { return g_last_error; }
+
+lq_status lq_pack(const int8_t* b_pm1, int32_t N, int32_t K, int32_t d, int32_t D,
+                  uint32_t* packed, lq_stream stream) {
+  clear_error();
+  if (!valid_code(K, d, D)) return fail(LQ_EINVAL, "invalid code sizes K=%d d=%d D=%d", K, d, D);
+  if (N < 0) return fail(LQ_EINVAL, "N = %d < 0", N);
+  if (N == 0) return LQ_OK;
+  if (!b_pm1 || !packed) return fail(LQ_EINVAL, "null pointer");
+  if (!aligned(packed, 16)) return fail(LQ_EINVAL, "packed is not 16-byte aligned");
+  cudaError_t e = lq::launch_pack(b_pm1, N, lifted_bits(K, d, D), row_stride_bytes(K, d, D) / 4,
+                                  packed, (cudaStream_t)stream);
+  return e == cudaSuccess ? LQ_OK : cuda_fail(e, "lq_pack");
+}
+
+lq_status lq_unpack(const uint32_t* packed, int32_t N, int32_t K, int32_t d, int32_t D,
+                    int8_t* b_pm1, lq_stream stream) {
+  clear_error();
+  if (!valid_code(K, d, D)) return fail(LQ_EINVAL, "invalid code sizes K=%d d=%d D=%d", K, d, D);
+  if (N < 0) return fail(LQ_EINVAL, "N = %d < 0", N);
+  if (N == 0) return LQ_OK;
+  if (!b_pm1 || !packed) return fail(LQ_EINVAL, "null pointer");
+  if (!aligned(packed, 16)) return fail(LQ_EINVAL, "packed is not 16-byte aligned");
+  cudaError_t e = lq::launch_unpack(packed, N, lifted_bits(K, d, D),
+                                    row_stride_bytes(K, d, D) / 4, b_pm1, (cudaStream_t)stream);
+  return e == cudaSuccess ? LQ_OK : cuda_fail(e, "lq_unpack");
+}
+
+lq_status lq_whiten(const void* x, lq_dtype xdt, int32_t batch, int32_t K,
+                    const lq_whiten_desc* T, float* xt, lq_stream stream) {
+  clear_error();
+  if (batch < 0 || batch > kMaxBatch) return fail(LQ_EINVAL, "batch = %d out of range", batch);
+  if (K < 1 || K > kMaxK) return fail(LQ_EINVAL, "K = %d out of range", K);
+  if (!valid_dtype(xdt)) return fail(LQ_EINVAL, "unknown x dtype %d", (int)xdt);
+  if (batch == 0) return LQ_OK;
+  if (!x || !xt) return fail(LQ_EINVAL, "null pointer");
+  if (!aligned(x, dtype_size(xdt)) || !aligned(xt, 4)) return fail(LQ_EINVAL, "misaligned x/xt");
+  lq::Whiten w;
+  lq_status st = make_whiten(T, K, &w);
+  if (st != LQ_OK) return st;
+  cudaError_t e = lq::launch_whiten(x, (int)xdt, batch, K, w, xt, (cudaStream_t)stream);
+  return e == cudaSuccess ? LQ_OK : cuda_fail(e, "lq_whiten");
+}
+
+lq_status lq_lift(const void* x, lq_dtype xdt, int32_t batch, int32_t K,
+                  const lq_whiten_desc* T, const float* M, int32_t d, int32_t D, float* z,
+                  lq_stream stream) {
+  clear_error();
+  if (!valid_code(K, d, D)) return fail(LQ_EINVAL, "invalid code sizes K=%d d=%d D=%d", K, d, D);
+  if (batch < 0 || batch > kMaxBatch) return fail(LQ_EINVAL, "batch = %d out of range", batch);
+  if (K > kMaxK) return fail(LQ_EINVAL, "K = %d out of range", K);
+  if (!valid_dtype(xdt)) return fail(LQ_EINVAL, "unknown x dtype %d", (int)xdt);
+  if (batch == 0) return LQ_OK;
+  if (!x || !M || !z) return fail(LQ_EINVAL, "null pointer");
+  if (!aligned(x, dtype_size(xdt)) || !aligned(M, 4) || !aligned(z, 4))
+    return fail(LQ_EINVAL, "misaligned x/M/z");
+  lq::Whiten w;
+  lq_status st = make_whiten(T, K, &w);
+  if (st != LQ_OK) return st;
+  cudaError_t e = lq::launch_lift_f32(x, (int)xdt, batch, K, w, M, d, D, z, nullptr, 0,
+                                      (cudaStream_t)stream);
+  return e == cudaSuccess ? LQ_OK : cuda_fail(e, "lq_lift");
+}
+
+size_t lq_gemm_workspace_bytes(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D) {
+  if (!valid_code(K, d, D) || batch < 1 || batch > kMaxBatch || N < 1 || K > kMaxK) return 0;
+  return layout_gemm(batch, K, N, d, D).total;
+}
+
+lq_status lq_gemm(const void* x, lq_dtype xdt, int32_t batch, const lq_whiten_desc* T,
+                  const uint32_t* packed, const float* M, const void* s, lq_dtype sdt,
+                  int32_t d, int32_t D, int32_t K, int32_t N, float* y, void* workspace,
+                  size_t workspace_bytes, lq_stream stream) {
+  clear_error();
+  if (!valid_code(K, d, D)) return fail(LQ_EINVAL, "invalid code sizes K=%d d=%d D=%d", K, d, D);
+  if (batch < 1 || batch > kMaxBatch) return fail(LQ_EINVAL, "batch = %d out of range", batch);
+  if (N < 1) return fail(LQ_EINVAL, "N = %d < 1", N);
+  if (K > kMaxK) return fail(LQ_EINVAL, "K = %d out of range", K);
+  if (!valid_dtype(xdt) || !valid_dtype(sdt)) return fail(LQ_EINVAL, "unknown dtype");
+  if (!x || !packed || !M || !s || !y || !workspace) return fail(LQ_EINVAL, "null pointer");
+  if (!aligned(packed, 16)) return fail(LQ_EINVAL, "packed is not 16-byte aligned");
+  if (!aligned(workspace, 256)) return fail(LQ_EINVAL, "workspace is not 256-byte aligned");
+  if (!aligned(x, dtype_size(xdt)) || !aligned(s, dtype_size(sdt)) || !aligned(M, 4) ||
+      !aligned(y, 4))
+    return fail(LQ_EINVAL, "misaligned x/s/M/y");
+  lq::Whiten w;
+  lq_status st = make_whiten(T, K, &w);
+  if (st != LQ_OK) return st;
+  const WsLayout lay = layout_gemm(batch, K, N, d, D);
+  if (workspace_bytes < lay.total)
+    return fail(LQ_EINVAL, "workspace of %zu bytes is smaller than the %zu bytes needed",
+                workspace_bytes, lay.total);
+  if (lay.gemv.ntiles > 65535 || lay.gemv.ntg > 65535)
+    return fail(LQ_EUNSUPPORTED, "N or batch too large for one launch");
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t cs = (cudaStream_t)stream;
+  const int64_t L = lifted_bits(K, d, D);
+  float* z = reinterpret_cast<float*>(ws + lay.z);
+  uint32_t* counters = reinterpret_cast<uint32_t*>(ws + lay.counters);
+  cudaError_t e = lq::launch_lift_f32(x, (int)xdt, batch, K, w, M, d, D, z, counters,
+                                      lay.gemv.ntg * lay.gemv.ntiles, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "lq_gemm (lift)");
+  e = lq::launch_gemv(lay.gemv, z, L, batch, packed, row_stride_bytes(K, d, D) / 4, N, s,
+                      (int)sdt, y, reinterpret_cast<float*>(ws + lay.partials), counters, cs);
+  return e == cudaSuccess ? LQ_OK : cuda_fail(e, "lq_gemm (gemv)");
+}
+
+lq_status lq_device_status(void* workspace, int32_t* code, lq_stream stream) {
+  clear_error();
+  if (!workspace || !code) return fail(LQ_EINVAL, "null pointer");
+  cudaStream_t cs = (cudaStream_t)stream;
+  uint32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, cs);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+  if (e != cudaSuccess) return cuda_fail(e, "lq_device_status");
+  *code = (int32_t)v;
+  if (v != 0) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyAsync(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice, cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+    if (e != cudaSuccess) return cuda_fail(e, "lq_device_status");
+    return (lq_status)v;
+  }
+  return LQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,63 @@
+// lq_internal.cuh -- declarations shared by the liblq CUDA sources (not part of the ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "liblq.h"
+
+namespace lq {
+
+// Parameters of the whitening T after host-side validation.
+struct Whiten {
+  const int8_t* sign;       // [K] or nullptr
+  const float* chan_scale;  // [K] or nullptr
+  int32_t block;            // 0 = identity, else a power of two dividing K
+  float inv_sqrt;           // 1/sqrt(block), computed on the host in double
+};
+
+// Byte offsets inside the caller's lq_gemm workspace.
+struct WsHeader {
+  uint32_t status;          // 0, or an lq_status recorded by a kernel
+  uint32_t reserved[63];
+};
+static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
+
+__device__ __forceinline__ float load_as_f32(const void* p, int dt, int64_t i) {
+  if (dt == LQ_F32) return static_cast<const float*>(p)[i];
+  if (dt == LQ_F16) return __half2float(static_cast<const __half*>(p)[i]);
+  return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+}
+
+// ---- launchers (host side); each returns cudaGetLastError() of its launch
+cudaError_t launch_pack(const int8_t* b, int32_t N, int64_t L, int64_t words, uint32_t* packed,
+                        cudaStream_t st);
+cudaError_t launch_unpack(const uint32_t* packed, int32_t N, int64_t L, int64_t words,
+                          int8_t* b, cudaStream_t st);
+cudaError_t launch_whiten(const void* x, int xdt, int32_t batch, int32_t K, Whiten T,
+                          float* xt, cudaStream_t st);
+// Fused whiten + lift into fp32 z [batch][G*D]. If zero_words > 0, the launch also clears
+// zero_ptr[0 .. zero_words) (the split-K counters of a following GEMV launch).
+cudaError_t launch_lift_f32(const void* x, int xdt, int32_t batch, int32_t K, Whiten T,
+                            const float* M, int32_t d, int32_t D, float* z, uint32_t* zero_ptr,
+                            int32_t zero_words, cudaStream_t st);
+
+// Plan of the small-batch GEMV over z (fp32, in global memory).
+struct GemvPlan {
+  int tb;        // tokens per CTA
+  int ntg;       // token groups
+  int sw;        // 32-bit words of a row per K-slice
+  int nsl;       // K-slices
+  int rt;        // rows per CTA
+  int ntiles;    // row tiles
+  size_t smem;   // dynamic shared memory per CTA
+};
+GemvPlan plan_gemv(int32_t batch, int64_t L, int32_t N);
+cudaError_t launch_gemv(const GemvPlan& p, const float* z, int64_t L, int32_t batch,
+                        const uint32_t* packed, int64_t row_words, int32_t N, const void* s,
+                        int sdt, float* y, float* partials, uint32_t* counters,
+                        cudaStream_t st);
+
+}  // namespace lq

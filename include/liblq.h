@@ -1,0 +1,148 @@
+/*
+ * liblq.h -- C ABI of the B200 (sm_100a) LiftQuant decode library.
+ *
+ * The operator (LiftQuant: Continuous Bit-Width LLM Quantization via Dimensional
+ * Lifting and Projection, sec. 3 intro and sec. 3.1; the romaanj.github.io review,
+ * "Method"):
+ *
+ *     y[t][n] = s[n] * sum_k W[n][k] * T(x[t])[k]
+ *     W[n][g*d + i] = sum_{j<D} M[i][j] * b[n][g][j],   b in {+1,-1}
+ *
+ * Each length-d block g of a weight row is stored as D sign bits b[n][g][.] and
+ * decoded through the d x D mapping matrix M, so a row of K inputs costs
+ * ceil(K/d) * D bits: the fractional bit-width D/d (24/10 = 2.4 bit). T is the
+ * whitening transform: a random +-1 diagonal (and optional per-channel scale)
+ * followed by the normalised Walsh-Hadamard transform on contiguous blocks.
+ * The library evaluates the lifted form y = s . (b . z) with
+ * z[t][g*D + j] = sum_i M[i][j] * T(x[t])[g*d + i], since b^T (M^T x) = (M b)^T x.
+ *
+ * Conventions for every entry point:
+ *   - All array arguments are DEVICE pointers owned by the caller, row-major and
+ *     dense. The library never allocates, frees, prints or exits.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls are
+ *     asynchronous with respect to the host; results are ready when the stream is.
+ *   - Arguments are checked on the host before anything is launched; a rejected
+ *     call launches nothing and returns LQ_EINVAL or LQ_EUNSUPPORTED.
+ *     lq_last_error() then holds a one-line reason (per host thread).
+ *   - A failed launch returns LQ_ECUDA. Device-side failures are recorded in the
+ *     workspace status word and read by lq_device_status().
+ *   - Calls that share a workspace must be ordered on one stream.
+ */
+#ifndef LIBLQ_H
+#define LIBLQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LQ_ABI_VERSION 1
+/* Stored-code format. Row n, block g, lifted coordinate j is bit q = g*D + j of
+ * the row; bit q is bit (q % 32) of 32-bit little-endian word q / 32 (equivalently
+ * bit q % 8 of byte q / 8); a set bit means b = -1 (it is the sign bit that flips
+ * z); each row is zero-padded to a multiple of 16 bytes. */
+#define LQ_FORMAT_V1 1
+/* Largest supported Hadamard block of T. */
+#define LQ_MAX_HADAMARD 4096
+/* Largest lifted dimension D per block (the pages' largest code is LQ-32/16). */
+#define LQ_MAX_D 32
+
+typedef enum lq_status {
+  LQ_OK = 0,
+  LQ_EINVAL = 1,        /* a null/misaligned pointer or an out-of-range size */
+  LQ_EUNSUPPORTED = 2,  /* valid, but not implemented (e.g. Hadamard block > LQ_MAX_HADAMARD) */
+  LQ_ECUDA = 3,         /* a CUDA launch or query failed */
+  LQ_ETIMEOUT = 4,      /* a bounded device-side wait expired (status word) */
+  LQ_EDEVICE = 5        /* a device-side check failed (status word) */
+} lq_status;
+
+typedef enum lq_dtype { LQ_F32 = 0, LQ_F16 = 1, LQ_BF16 = 2 } lq_dtype;
+
+typedef void* lq_stream; /* a cudaStream_t */
+
+#if defined(__GNUC__)
+#define LQ_API __attribute__((visibility("default")))
+#else
+#define LQ_API
+#endif
+
+/* The whitening transform T: xt = H_Bh (sign . chan_scale . x) / sqrt(Bh) on each
+ * contiguous block of Bh inputs, H in Sylvester (natural) order,
+ * H[i][j] = (-1)^popcount(i & j). A NULL descriptor, or block == 0, is the identity. */
+typedef struct lq_whiten_desc {
+  const int8_t* sign;       /* [K] device, entries +1/-1; NULL = all +1 */
+  const float* chan_scale;  /* [K] device; NULL = all 1 */
+  int32_t block;            /* Bh: 0 (identity) or a power of two <= LQ_MAX_HADAMARD dividing K */
+} lq_whiten_desc;
+
+/* ABI version (LQ_ABI_VERSION) of the loaded library. */
+LQ_API int32_t lq_abi_version(void);
+
+/* Stored bits per row, ceil(K/d) * D (the paper's rate D/d when d divides K).
+ * Returns -1 if K < 1, d < 1, D < d or D > LQ_MAX_D. */
+LQ_API int64_t lq_lifted_bits(int32_t K, int32_t d, int32_t D);
+
+/* Bytes per stored row: the lifted bits rounded up to a multiple of 16 bytes.
+ * Returns -1 on invalid sizes (as lq_lifted_bits). */
+LQ_API int64_t lq_row_stride_bytes(int32_t K, int32_t d, int32_t D);
+
+/* Pack sign codes into LQ_FORMAT_V1 rows (offline step, paper sec. 3.1: w ~= M w_q).
+ *   b_pm1  [N][ceil(K/d)*D] int8: entries < 0 are stored as -1, all others as +1.
+ *   packed [N][lq_row_stride_bytes/4] uint32, 16-byte aligned; padding bits are written as 0.
+ * Errors: LQ_EINVAL for null pointers, misalignment or invalid sizes (N >= 0; N = 0 is a no-op). */
+LQ_API lq_status lq_pack(const int8_t* b_pm1, int32_t N, int32_t K, int32_t d, int32_t D,
+                  uint32_t* packed, lq_stream stream);
+
+/* Inverse of lq_pack: packed rows -> [N][ceil(K/d)*D] int8 of +1/-1. Padding is ignored. */
+LQ_API lq_status lq_unpack(const uint32_t* packed, int32_t N, int32_t K, int32_t d, int32_t D,
+                    int8_t* b_pm1, lq_stream stream);
+
+/* Whitening alone: xt = T(x) (review, "Method": Hadamard mixing plus scalings).
+ *   x  [batch][K] of dtype xdt;  xt [batch][K] float32.
+ * Errors: LQ_EINVAL (null pointers, batch < 0, K < 1, bad block), LQ_EUNSUPPORTED
+ * (block > LQ_MAX_HADAMARD). */
+LQ_API lq_status lq_whiten(const void* x, lq_dtype xdt, int32_t batch, int32_t K,
+                    const lq_whiten_desc* T, float* xt, lq_stream stream);
+
+/* Whitening fused with the lift: z[t][g*D + j] = sum_{i<d} M[i][j] * T(x[t])[g*d + i],
+ * with T(x) zero beyond K (review, "Method": T* = lift composed with T).
+ *   M [d][D] float32 row-major; z [batch][ceil(K/d)*D] float32. */
+LQ_API lq_status lq_lift(const void* x, lq_dtype xdt, int32_t batch, int32_t K,
+                  const lq_whiten_desc* T, const float* M, int32_t d, int32_t D, float* z,
+                  lq_stream stream);
+
+/* Workspace bytes lq_gemm needs for this shape (0 on invalid sizes). */
+LQ_API size_t lq_gemm_workspace_bytes(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D);
+
+/* The decode operator, y = s . (W T(x)) (paper sec. 3 intro: o = diag(s) W (M T a);
+ * review: diag(s) W_q (T* a)).
+ *   x       [batch][K] of dtype xdt (f32, f16 or bf16)
+ *   packed  [N][lq_row_stride_bytes/4] uint32 LQ_FORMAT_V1 rows, 16-byte aligned
+ *   M       [d][D] float32;  s [N] of dtype sdt;  y [batch][N] float32 (overwritten)
+ *   workspace: lq_gemm_workspace_bytes(...) bytes, 256-byte aligned, caller-owned.
+ *     It must be zero-filled before its first use; every call leaves it ready for the next.
+ * Accumulation is fp32 in a fixed order: the result does not depend on timing.
+ * Errors: LQ_EINVAL (null or misaligned pointers, batch < 1, N < 1, bad sizes,
+ * workspace too small), LQ_EUNSUPPORTED (block > LQ_MAX_HADAMARD), LQ_ECUDA. */
+LQ_API lq_status lq_gemm(const void* x, lq_dtype xdt, int32_t batch, const lq_whiten_desc* T,
+                  const uint32_t* packed, const float* M, const void* s, lq_dtype sdt,
+                  int32_t d, int32_t D, int32_t K, int32_t N, float* y, void* workspace,
+                  size_t workspace_bytes, lq_stream stream);
+
+/* Synchronise `stream`, then read the workspace status word into *code (0 = no device-side
+ * failure) and clear it. Returns LQ_OK, or the lq_status that the word records. */
+LQ_API lq_status lq_device_status(void* workspace, int32_t* code, lq_stream stream);
+
+/* Static text for a status code. */
+LQ_API const char* lq_status_string(lq_status status);
+
+/* Reason for the last rejected call on this host thread ("" if none). */
+LQ_API const char* lq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBLQ_H */

@@ -1,0 +1,108 @@
+"""liblq.so loads, exports every entry point that include/liblq.h declares, and its host-side
+logic (sizes, argument checks) agrees with the oracle. No GPU is used: every call below
+returns before any CUDA work."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import fractional_bit_weight_b200 as lq
+from fractional_bit_weight_b200 import build as lqbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "liblq.h")
+
+
+def declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^LQ_API\s+[^(]*?\b(lq_\w+)\s*\(", text, re.M)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    lqbuild.build()
+    return lq.lib()
+
+
+def test_header_declares_entry_points():
+    names = declared()
+    for required in ("lq_pack", "lq_whiten", "lq_gemm"):
+        assert required in names
+    assert set(names) == set(lq.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared():
+        assert hasattr(L, name), name
+    out = os.popen(f"nm -D --defined-only {lq.LIB_PATH}").read()
+    exported = set(re.findall(r"\bT (lq_\w+)", out))
+    assert set(declared()) <= exported
+    assert exported <= set(declared()), exported - set(declared())
+
+
+def test_sizes_match_oracle(L, orc):
+    assert lq.abi_version() == 1
+    for K, d, D in [(256, 2, 5), (4096, 10, 24), (28672, 10, 24), (8192, 3, 8), (7, 3, 5),
+                    (1, 1, 1), (8192, 16, 32), (100, 10, 25)]:
+        assert lq.lifted_bits(K, d, D) == orc.lifted_bits(K, d, D)
+        assert lq.row_stride_bytes(K, d, D) == orc.row_bytes(K, d, D)
+    for K, d, D in [(0, 1, 1), (10, 0, 1), (10, 5, 4), (10, 8, 33)]:
+        assert lq.lifted_bits(K, d, D) == -1
+        assert lq.row_stride_bytes(K, d, D) == -1
+
+
+def test_workspace_bytes(L):
+    assert lq.gemm_workspace_bytes(1, 4096, 4096, 10, 24) > 0
+    assert lq.gemm_workspace_bytes(1, 4096, 4096, 10, 24) % 256 == 0
+    assert lq.gemm_workspace_bytes(0, 4096, 4096, 10, 24) == 0
+    assert lq.gemm_workspace_bytes(1, 4096, 0, 10, 24) == 0
+    assert lq.gemm_workspace_bytes(1, 4096, 4096, 10, 33) == 0
+
+
+def _ptr(v):
+    return ctypes.c_void_p(v)
+
+
+def test_argument_checks_without_gpu(L):
+    fake = _ptr(0x10000)       # aligned, never dereferenced: every call below is rejected
+    odd = _ptr(0x10004)
+    S = None
+    assert L.lq_pack(None, 4, 16, 2, 4, fake, S) == lq.LQ_EINVAL
+    assert L.lq_pack(fake, 4, 16, 2, 4, odd, S) == lq.LQ_EINVAL      # packed misaligned
+    assert L.lq_pack(fake, -1, 16, 2, 4, fake, S) == lq.LQ_EINVAL
+    assert L.lq_pack(fake, 0, 16, 2, 4, fake, S) == lq.LQ_OK         # N = 0: no work
+    assert L.lq_pack(fake, 4, 16, 5, 4, fake, S) == lq.LQ_EINVAL     # D < d
+    assert "D" in L.lq_last_error().decode() or "invalid" in L.lq_last_error().decode()
+    assert L.lq_unpack(fake, 4, 16, 2, 40, fake, S) == lq.LQ_EINVAL  # D > 32
+
+    bad = lq.WhitenDesc(None, None, 3)
+    assert L.lq_whiten(fake, 0, 2, 12, ctypes.byref(bad), fake, S) == lq.LQ_EINVAL
+    big = lq.WhitenDesc(None, None, 8192)
+    assert L.lq_whiten(fake, 0, 1, 8192, ctypes.byref(big), fake, S) == lq.LQ_EUNSUPPORTED
+    nodiv = lq.WhitenDesc(None, None, 256)
+    assert L.lq_whiten(fake, 0, 1, 300, ctypes.byref(nodiv), fake, S) == lq.LQ_EINVAL
+    assert L.lq_whiten(fake, 7, 1, 256, None, fake, S) == lq.LQ_EINVAL   # unknown dtype
+
+    args = dict(x=fake, xdt=2, batch=1, T=None, packed=fake, M=fake, s=fake, sdt=1, d=10, D=24,
+                K=4096, N=4096, y=fake, ws=fake, wsb=1 << 30)
+
+    def gemm(**kw):
+        a = dict(args, **kw)
+        return L.lq_gemm(a["x"], a["xdt"], a["batch"], a["T"], a["packed"], a["M"], a["s"],
+                         a["sdt"], a["d"], a["D"], a["K"], a["N"], a["y"], a["ws"], a["wsb"], S)
+
+    assert gemm(batch=0) == lq.LQ_EINVAL
+    assert gemm(N=0) == lq.LQ_EINVAL
+    assert gemm(packed=None) == lq.LQ_EINVAL
+    assert gemm(packed=_ptr(0x10008)) == lq.LQ_EINVAL
+    assert gemm(ws=_ptr(0x10010)) == lq.LQ_EINVAL                      # not 256-aligned
+    assert gemm(wsb=16) == lq.LQ_EINVAL
+    assert "workspace" in L.lq_last_error().decode()
+    assert gemm(T=ctypes.byref(lq.WhitenDesc(None, None, 3000))) == lq.LQ_EINVAL
+    assert gemm(x=_ptr(0x10001)) == lq.LQ_EINVAL                       # bf16 x misaligned
+    assert gemm(D=8) == lq.LQ_EINVAL
+    code = ctypes.c_int32(0)
+    assert L.lq_device_status(None, ctypes.byref(code), S) == lq.LQ_EINVAL
+    for st in range(6):
+        assert L.lq_status_string(st)
