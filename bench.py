@@ -231,25 +231,53 @@ def _x_tensor(layer):
     return torch.from_numpy(np.ascontiguousarray(layer.x_raw))
 
 
-def kernels_per_step():
-    return 2      # lift prologue + contraction
+def kernels_per_step(batch):
+    """Kernels one lq_gemm call launches: the fused int8 GEMV (batch <= 8), else the lift
+    prologue plus the fp32 GEMV."""
+    return 1 if batch <= 8 else 2
 
 
-def time_steps(fn, steps, warmup, ws):
+def time_steps(fn, steps, warmup, ws, graph_block=None):
+    """Device time of exactly `steps` calls of fn(i), after `warmup` untimed calls.
+
+    With graph_block, the calls are captured into CUDA graphs of graph_block steps (plus one
+    graph for the remainder) and replayed, so host launch overhead stays out of the timing."""
     for i in range(warmup):
         fn(i)
     torch.cuda.synchronize()
+    graphs = []
+    if graph_block:
+        gb = max(1, min(graph_block, steps))
+        sizes = [gb] * (steps // gb) + ([steps % gb] if steps % gb else [])
+        cache = {}
+        base = warmup
+        for n in sizes:
+            if n not in cache:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    for i in range(n):
+                        fn(base + i)
+                cache[n] = g
+            graphs.append(cache[n])
+        for g in cache.values():          # warm the graphs
+            g.replay()
+        torch.cuda.synchronize()
     barrier(ws)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for i in range(steps):
-        fn(warmup + i)
+    if graphs:
+        for g in graphs:
+            g.replay()
+    else:
+        for i in range(steps):
+            fn(warmup + i)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(ws)
     torch.cuda.synchronize()
+    del graphs
     return e0.elapsed_time(e1) / 1e3   # seconds
 
 
@@ -301,7 +329,7 @@ def main():
     peaks, peak_src = measured_peaks()
 
     with ClockSampler(local) as clk:
-        secs = time_steps(wl.step, args.steps, args.warmup, ws)
+        secs = time_steps(wl.step, args.steps, args.warmup, ws, graph_block=wl.ncopies)
     secs = max_over_ranks(secs, ws)
     per_step = secs / args.steps
 
@@ -335,7 +363,8 @@ def main():
                    "l2": f"rotating {wl.ncopies} copies of the packed weights "
                          f"({wl.ncopies * wl.stored_bytes / 1e6:.0f} MB > L2)"},
         "roofline": roof,
-        "gpu_launches": kernels_per_step() * args.steps,
+        "gpu_launches": kernels_per_step(wl.batch) * args.steps,
+        "timing": "CUDA graphs of the steps, replayed; CUDA events on the launching stream",
         "clocks": clk.summary(),
     }
     if kind == "gemv":

@@ -70,24 +70,37 @@ lq_status make_whiten(const lq_whiten_desc* T, int32_t K, lq::Whiten* out) {
 
 // Workspace layout of lq_gemm (byte offsets, all 256-aligned).
 struct WsLayout {
-  size_t counters;   // uint32 [ntg * ntiles]
-  size_t z;          // float  [batch][L]
-  size_t partials;   // float  [nsl][batch][N]
+  int path;          // 0: int8 tensor-core GEMV (batch <= 8); 1: fp32 GEMV over z
+  size_t counters;   // uint32 completion counters of the split-K reduction
+  size_t z;          // float z [batch][L] (path 1)
+  size_t partials;   // float [slices][batch][N]
   size_t total;
   lq::GemvPlan gemv;
+  lq::G8Plan g8;
 };
 
-WsLayout layout_gemm(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D) {
+WsLayout layout_gemm(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D, int32_t Bh) {
   WsLayout w{};
   const int64_t L = lifted_bits(K, d, D);
-  w.gemv = lq::plan_gemv(batch, L, N);
+  w.g8 = lq::plan_gemv_i8(batch, L, N, K, d, D, Bh);
+  w.path = w.g8.ok ? 0 : 1;
+  size_t ncounters = 0, npartials = 0, nz = 0;
+  if (w.path == 0) {
+    ncounters = (size_t)w.g8.R;
+    npartials = w.g8.S > 1 ? (size_t)w.g8.S * batch * N : 0;
+  } else {
+    w.gemv = lq::plan_gemv(batch, L, N);
+    ncounters = (size_t)w.gemv.ntg * w.gemv.ntiles;
+    npartials = w.gemv.nsl > 1 ? (size_t)w.gemv.nsl * batch * N : 0;
+    nz = (size_t)batch * L;
+  }
   size_t off = sizeof(lq::WsHeader);
   w.counters = off;
-  off = round_up(off + (size_t)w.gemv.ntg * w.gemv.ntiles * sizeof(uint32_t), 256);
+  off = round_up(off + ncounters * sizeof(uint32_t), 256);
   w.z = off;
-  off = round_up(off + (size_t)batch * L * sizeof(float), 256);
+  off = round_up(off + nz * sizeof(float), 256);
   w.partials = off;
-  if (w.gemv.nsl > 1) off = round_up(off + (size_t)w.gemv.nsl * batch * N * sizeof(float), 256);
+  off = round_up(off + npartials * sizeof(float), 256);
   w.total = off;
   return w;
 }
@@ -187,7 +200,11 @@ lq_status lq_lift(const void* x, lq_dtype xdt, int32_t batch, int32_t K,
 
 size_t lq_gemm_workspace_bytes(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D) {
   if (!valid_code(K, d, D) || batch < 1 || batch > kMaxBatch || N < 1 || K > kMaxK) return 0;
-  return layout_gemm(batch, K, N, d, D).total;
+  // the plan (and so the workspace) depends on the Hadamard block; return the largest
+  size_t best = 0;
+  for (int32_t Bh = 0; Bh <= LQ_MAX_HADAMARD; Bh = Bh ? 2 * Bh : 1)
+    best = std::max(best, layout_gemm(batch, K, N, d, D, Bh).total);
+  return best;
 }
 
 lq_status lq_gemm(const void* x, lq_dtype xdt, int32_t batch, const lq_whiten_desc* T,
@@ -209,22 +226,29 @@ lq_status lq_gemm(const void* x, lq_dtype xdt, int32_t batch, const lq_whiten_de
   lq::Whiten w;
   lq_status st = make_whiten(T, K, &w);
   if (st != LQ_OK) return st;
-  const WsLayout lay = layout_gemm(batch, K, N, d, D);
+  const WsLayout lay = layout_gemm(batch, K, N, d, D, w.block);
   if (workspace_bytes < lay.total)
     return fail(LQ_EINVAL, "workspace of %zu bytes is smaller than the %zu bytes needed",
                 workspace_bytes, lay.total);
-  if (lay.gemv.ntiles > 65535 || lay.gemv.ntg > 65535)
-    return fail(LQ_EUNSUPPORTED, "N or batch too large for one launch");
   char* ws = static_cast<char*>(workspace);
   cudaStream_t cs = (cudaStream_t)stream;
   const int64_t L = lifted_bits(K, d, D);
-  float* z = reinterpret_cast<float*>(ws + lay.z);
   uint32_t* counters = reinterpret_cast<uint32_t*>(ws + lay.counters);
+  float* partials = reinterpret_cast<float*>(ws + lay.partials);
+  if (lay.path == 0) {
+    cudaError_t e = lq::launch_gemv_i8(lay.g8, x, (int)xdt, batch, K, w, M, d, D, L, packed,
+                                       row_stride_bytes(K, d, D), N, s, (int)sdt, y, partials,
+                                       counters, cs);
+    return e == cudaSuccess ? LQ_OK : cuda_fail(e, "lq_gemm (int8 gemv)");
+  }
+  if (lay.gemv.ntiles > 65535 || lay.gemv.ntg > 65535)
+    return fail(LQ_EUNSUPPORTED, "N or batch too large for one launch");
+  float* z = reinterpret_cast<float*>(ws + lay.z);
   cudaError_t e = lq::launch_lift_f32(x, (int)xdt, batch, K, w, M, d, D, z, counters,
                                       lay.gemv.ntg * lay.gemv.ntiles, cs);
   if (e != cudaSuccess) return cuda_fail(e, "lq_gemm (lift)");
   e = lq::launch_gemv(lay.gemv, z, L, batch, packed, row_stride_bytes(K, d, D) / 4, N, s,
-                      (int)sdt, y, reinterpret_cast<float*>(ws + lay.partials), counters, cs);
+                      (int)sdt, y, partials, counters, cs);
   return e == cudaSuccess ? LQ_OK : cuda_fail(e, "lq_gemm (gemv)");
 }
 

@@ -117,12 +117,9 @@ static cudaError_t launch_tb(const GemvPlan& p, const float* z, int64_t L, int32
                              const uint32_t* packed, int64_t row_words, int32_t N,
                              const void* s, int sdt, float* y, float* partials,
                              uint32_t* counters, cudaStream_t st) {
-  if (p.smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_xor_kernel<TB>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)p.smem);
-    if (e != cudaSuccess) return e;
-  }
+  static int smem_set[64];
+  cudaError_t e = ensure_smem((const void*)gemv_xor_kernel<TB>, p.smem, smem_set);
+  if (e != cudaSuccess) return e;
   dim3 grid(p.nsl, p.ntiles, p.ntg);
   gemv_xor_kernel<TB><<<grid, kGemvThreads, p.smem, st>>>(z, L, batch, packed, row_words, N,
                                                           s, sdt, y, p.sw, p.nsl, p.rt,

@@ -1,0 +1,567 @@
+// lq_gemv_i8.cu -- decode GEMV for small batches (batch <= 8), one kernel per call.
+//
+// y[t][n] = s[n] * sum_q b[n][q] z[t][q] with b in {+1,-1}, z = lift(T(x[t]))
+// (paper sec. 3 intro: o = diag(s) W (M T a); review "Method": an INT1 x FP product plus small
+// linear maps, with no lookup table). With b = 1 - 2*bit,
+//     sum_q b_q z_q = sum_q z_q - 2 * sum_{q: bit_q = 1} z_q,
+// so each row needs only the subset sum of z over its set bits.
+//
+// The lifted dimension is cut into 512-bit chunks and the chunks into S slices; the grid is
+// S slices x R row ranges, one CTA each (one CTA per SM). A CTA:
+//  1. starts streaming its first stored bits into registers;
+//  2. prologue, in shared memory: whitens the Hadamard blocks that feed its slice (one warp per
+//     block: the first butterfly stages in registers, the rest with lane shuffles), lifts them,
+//     z = M^T xt per block of d inputs (one value per thread at a time), picks a power-of-two
+//     scale S from max|z| of each chunk, and splits z*S*2^-p, p = q mod 8, into four int8
+//     planes (base 254) written in the register layout of the B operand of mma.m16n8k32
+//     (8 columns = 2 tokens x 4 planes), with the chunk's column weights -2*254^-plane/S and
+//     its sum of z;
+//  3. main loop: the (32-row tile pair, chunk) items of its rows, pair-major, in 16 equal
+//     contiguous runs, one per warp. A 32-bit word of stored bits becomes an int8 A operand
+//     with one AND, (w & 0x01010101 << p): bit p of each byte as 0 or 2^p; the B entries carry
+//     2^-p, so all eight bit positions accumulate into one int32 set per item, scaled to fp32
+//     by the chunk's column weights;
+//  4. warps park the fp32 partial of every pair they touched in their own shared-memory slot;
+//     the slots are summed in warp order. With S > 1 each CTA writes its slice's partial and
+//     the last CTA of a row range to finish adds the slices in slice order and applies s.
+// Every CTA of a slice computes identical fragments, and all sums run in a fixed order, so the
+// result does not depend on timing.
+#include "lq_device.cuh"
+
+namespace lq {
+
+namespace g8 {
+constexpr int kWarps = 16;
+constexpr int kThreads = kWarps * 32;
+constexpr int kFragBytesPerChunk = 16 * 32 * 8;  // 16 MMAs (2 k-halves x 8 bit positions)
+constexpr int kMaxTokens = 8;
+constexpr int kPrefetch = 4;                      // items of stored bits in flight per warp
+constexpr int kMaxPairsPerWarp = 3;               // fp32 partial slots per warp
+constexpr int kSlotFloatsPerNT = 2 * 32 * 4;      // one tile pair: 2 tiles x 32 lanes x 4 regs
+}  // namespace g8
+
+struct G8Params {
+  const void* x;
+  int xdt;
+  int batch;
+  int K;
+  Whiten T;
+  const float* M;
+  int d;
+  int D;
+  int64_t L;
+  const uint8_t* packed;
+  int64_t row_bytes;
+  int N;
+  const void* s;
+  int sdt;
+  float* y;
+  float* partials;      // [S][batch][N] when S > 1
+  uint32_t* counters;   // [R] when S > 1
+  int nchunk;           // 512-bit chunks per row
+  int sc;               // chunks per slice
+  int S;                // slices
+  int R;                // row ranges
+  int xs_floats;        // whitening scratch per token
+};
+
+__device__ __forceinline__ void imma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint4 ldg_stream_v4(const uint8_t* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// four int8 planes of base 254: a ~= P0 + P1/254 + P2/254^2 + P3/254^3 (|a| < 64)
+__device__ __forceinline__ void planes4(float a, int (&P)[4]) {
+  P[0] = __float2int_rn(a);
+  float r = (a - (float)P[0]) * 254.f;
+  P[1] = __float2int_rn(r);
+  r = (r - (float)P[1]) * 254.f;
+  P[2] = __float2int_rn(r);
+  r = (r - (float)P[2]) * 254.f;
+  P[3] = __float2int_rn(r);
+}
+
+template <int NT>
+__global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params P) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ float s_sumz[g8::kMaxTokens];
+  __shared__ float s_scale[16 * g8::kMaxTokens];   // per (chunk, token); chunks per slice <= 16
+  __shared__ int s_pfirst[g8::kWarps];
+  __shared__ int s_last;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int sl = blockIdx.x % P.S, ri = blockIdx.x / P.S;
+  const int c0 = sl * P.sc;
+  const int nc = min(P.sc, P.nchunk - c0);
+  const int ra = (int)((int64_t)ri * P.N / P.R);
+  const int rb = (int)((int64_t)(ri + 1) * P.N / P.R);
+  const int npair = (rb - ra + 31) / 32;
+  const int items = npair * nc;
+  const int i0 = (int)((int64_t)warp * items / g8::kWarps);
+  const int i1 = (int)((int64_t)(warp + 1) * items / g8::kWarps);
+  const int n = i1 - i0;
+  const int pfirst = i0 / nc;
+
+  constexpr int kSlotFloats = g8::kSlotFloatsPerNT * NT;
+  uint2* sfr = reinterpret_cast<uint2*>(smem);                                  // [NT][sc][16][32]
+  float* slots = reinterpret_cast<float*>(smem + (size_t)NT * P.sc * g8::kFragBytesPerChunk);
+  float* xs = slots + (size_t)g8::kWarps * g8::kMaxPairsPerWarp * kSlotFloats;  // [batch][xs_floats]
+  float* Ms = xs + (size_t)P.batch * P.xs_floats;                               // [d][D]
+  float* wts = Ms + g8::kMaxTokens * 128;                                       // [sc][NT][8]
+  float* csum = wts + (size_t)P.sc * NT * 8;                                    // [sc][batch]
+
+  // ---- 1. start streaming: item i = (pair i / nc, chunk c0 + i % nc)
+  const int64_t last_off = P.row_bytes - 16;
+  int lpr = pfirst, lc = i0 - pfirst * nc;       // position of the next item to load
+  const uint8_t* rowp[4];
+  bool lhasB = false;
+  auto set_rows = [&](int pr) {
+    const int r = ra + pr * 32 + g;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int row = r + 8 * k;
+      rowp[k] = P.packed + (int64_t)(row < rb ? row : ra) * P.row_bytes + 16 * t;
+    }
+    lhasB = ra + pr * 32 + 16 < rb;
+  };
+  auto load_next = [&](uint4 (&u)[4]) {
+    int64_t off = (int64_t)(c0 + lc) * 64;
+    off = off + 16 * t > last_off ? last_off - 16 * t : off;   // last chunk: stay in the row
+    u[0] = ldg_stream_v4(rowp[0] + off);
+    u[1] = ldg_stream_v4(rowp[1] + off);
+    if (lhasB) {
+      u[2] = ldg_stream_v4(rowp[2] + off);
+      u[3] = ldg_stream_v4(rowp[3] + off);
+    }
+    if (++lc == nc) {
+      lc = 0;
+      if (++lpr < npair) set_rows(lpr);
+    }
+  };
+  if (n > 0) set_rows(lpr);
+  uint4 q[g8::kPrefetch][4];
+#pragma unroll
+  for (int k = 0; k < g8::kPrefetch; ++k)
+    if (k < n) load_next(q[k]);
+
+  // ---- 2. prologue: this slice's fragments, column weights and chunk sums
+  if (lane == 0) s_pfirst[warp] = pfirst;
+  for (int i = tid; i < P.d * P.D; i += g8::kThreads) Ms[i] = P.M[i];
+  const int64_t q0 = (int64_t)c0 * 512;
+  const int64_t q1 = min((int64_t)(c0 + nc) * 512, P.L);
+  const int g_lo = (int)(q0 / P.D), g_hi = (int)((q1 - 1) / P.D);
+  const int k0 = g_lo * P.d;
+  const int k1 = min((g_hi + 1) * P.d, P.K);
+  const int Bh = P.T.block;
+  int base = k0, span = k1 - k0;
+  if (Bh > 0) {
+    const int blk0 = k0 / Bh;
+    base = blk0 * Bh;
+    span = ((k1 + Bh - 1) / Bh - blk0) * Bh;
+  }
+  if (Bh >= 32 && Bh <= 256) {
+    // one warp per (token, block); lane l holds elements [E*l, E*l + E)
+    const int E = Bh >> 5;
+    const int nblk = span / Bh;
+    for (int task = warp; task < P.batch * nblk; task += g8::kWarps) {
+      const int tok = task / nblk, b = task - tok * nblk;
+      float v[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        if (r < E) {
+          const int k = base + b * Bh + E * lane + r;
+          float a = load_as_f32(P.x, P.xdt, (int64_t)tok * P.K + k);
+          if (P.T.chan_scale) a *= P.T.chan_scale[k];
+          if (P.T.sign && P.T.sign[k] < 0) a = -a;
+          v[r] = a;
+        }
+      }
+#pragma unroll
+      for (int h = 1; h < 8; h <<= 1)
+        if (h < E)
+#pragma unroll
+          for (int r = 0; r < 8; ++r)
+            if (r < E && (r & h) == 0) {
+              const float a = v[r], c2 = v[r + h];
+              v[r] = a + c2;
+              v[r + h] = a - c2;
+            }
+#pragma unroll
+      for (int m = 1; m < 32; m <<= 1) {
+        const bool upper = (lane & m) != 0;
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+          if (r < E) {
+            const float o = __shfl_xor_sync(0xffffffffu, v[r], m);
+            v[r] = upper ? o - v[r] : v[r] + o;
+          }
+      }
+      float* xt = xs + tok * P.xs_floats + b * Bh + E * lane;
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (r < E) xt[r] = v[r];
+    }
+    __syncthreads();
+  } else {
+    for (int e = tid; e < P.batch * span; e += g8::kThreads) {
+      const int tok = e / span, i = e - tok * span;
+      const int k = base + i;
+      float a = 0.f;
+      if (k < P.K) {
+        a = load_as_f32(P.x, P.xdt, (int64_t)tok * P.K + k);
+        if (Bh > 0) {
+          if (P.T.chan_scale) a *= P.T.chan_scale[k];
+          if (P.T.sign && P.T.sign[k] < 0) a = -a;
+        }
+      }
+      xs[tok * P.xs_floats + i] = a;
+    }
+    __syncthreads();
+    if (Bh > 1) {
+      const int half = span / 2;
+      for (int h = 1; h < Bh; h <<= 1) {
+        for (int pp = tid; pp < P.batch * half; pp += g8::kThreads) {
+          const int tok = pp / half, pi = pp - tok * half;
+          const int lo = pi & (h - 1);
+          const int i = ((pi - lo) << 1) | lo;
+          float* xt = xs + tok * P.xs_floats;
+          const float a = xt[i], c2 = xt[i + h];
+          xt[i] = a + c2;
+          xt[i + h] = a - c2;
+        }
+        __syncthreads();
+      }
+    }
+  }
+  // lift: every thread computes whole values z[e] of the slice (e = 512 * chunk + offset),
+  // all tokens, into shared memory (the lift runs over the d inputs of the value's block)
+  float* zs = slots;   // the partial slots are free until the main loop
+  const int nq = (int)(q1 - q0);
+  for (int tok = 0; tok < P.batch; ++tok) {
+    const float* xt = xs + tok * P.xs_floats;
+    for (int e = tid; e < nc * 512; e += g8::kThreads) {
+      float acc = 0.f;
+      if (e < nq) {
+        const int qi = (int)(q0 + e);
+        const int gg = qi / P.D;
+        const int jj = qi - gg * P.D;
+        const float* xg = xt + (gg * P.d - base);
+        const float* mj = Ms + jj;
+        const int dv = min(P.d, P.K - gg * P.d);   // inputs past K are zero
+        for (int ii = 0; ii < dv; ++ii) acc = fmaf(mj[ii * P.D], xg[ii], acc);
+        acc *= P.T.inv_sqrt;
+      }
+      zs[tok * (P.sc * 512) + e] = acc;
+    }
+  }
+  __syncthreads();
+  // per (chunk, token): max|z| -> power-of-two scale, and the sum of z; one warp each
+  for (int task = warp; task < nc * P.batch; task += g8::kWarps) {
+    const int cl = task / P.batch, tok = task - cl * P.batch;
+    const float* zc = zs + tok * (P.sc * 512) + cl * 512;
+    float lmax = 0.f, lsum = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float v = zc[lane + 32 * i];
+      lmax = fmaxf(lmax, fabsf(v));
+      lsum += v;
+    }
+    const float m = warp_max(lmax);
+    const float su = warp_sum(lsum);
+    if (lane == 0) {
+      int ex = 0;
+      frexpf(m, &ex);                                         // m = f * 2^ex, f in [0.5, 1)
+      const float Ssc = m > 0.f ? ldexpf(1.f, 6 - ex) : 1.f;  // |z| * S < 64
+      csum[cl * P.batch + tok] = su;
+      const int nt = tok >> 1, cb = (tok & 1) * 4;
+      float w = -2.f / Ssc;
+      for (int pl = 0; pl < 4; ++pl) {
+        wts[(cl * NT + nt) * 8 + cb + pl] = w;
+        w *= (float)(1.0 / 254.0);
+      }
+      s_scale[cl * g8::kMaxTokens + tok] = Ssc;
+    }
+  }
+  // weights of unused token columns
+  for (int i = tid; i < nc * NT * 8; i += g8::kThreads) {
+    const int col = i & 7, nt = (i >> 3) % NT;
+    if (nt * 2 + (col >> 2) >= P.batch) wts[i] = 0.f;
+  }
+  __syncthreads();
+  // quantise: a group (chunk, token slot, tt, j, h, p) is 4 values e0 + 8*i, i = 0..3, which
+  // fill one 32-bit word per plane: word (j*8 + p)*64 + 2*(4*col + tt) + h of the chunk
+  for (int gi = tid; gi < nc * 2 * NT * 128; gi += g8::kThreads) {
+    const int cl = gi / (2 * NT * 128);
+    const int rem = gi - cl * (2 * NT * 128);
+    const int tok = rem >> 7, grp = rem & 127;
+    const int tt = grp >> 5, jl = (grp >> 4) & 1, hl = (grp >> 3) & 1, pl8 = grp & 7;
+    const int nt = tok >> 1, cb = (tok & 1) * 4;
+    uint32_t w4[4] = {0u, 0u, 0u, 0u};
+    if (tok < P.batch) {
+      const float Sp = s_scale[cl * g8::kMaxTokens + tok] * __int_as_float((127 - pl8) << 23);
+      const float* zc = zs + tok * (P.sc * 512) + cl * 512 + 128 * tt + 64 * jl + 32 * hl + pl8;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        int Pq[4];
+        planes4(zc[8 * i] * Sp, Pq);
+#pragma unroll
+        for (int pl = 0; pl < 4; ++pl) w4[pl] |= ((uint32_t)Pq[pl] & 0xffu) << (8 * i);
+      }
+    }
+    uint32_t* fw = reinterpret_cast<uint32_t*>(sfr) + ((size_t)nt * P.sc + cl) * (g8::kFragBytesPerChunk / 4);
+#pragma unroll
+    for (int pl = 0; pl < 4; ++pl) fw[(jl * 8 + pl8) * 64 + 2 * (4 * (cb + pl) + tt) + hl] = w4[pl];
+  }
+  __syncthreads();
+  if (tid < P.batch) {
+    float a = 0.f;
+    for (int c = 0; c < nc; ++c) a += csum[c * P.batch + tid];
+    s_sumz[tid] = a;
+  }
+
+  // ---- 3. main loop
+  float accf[2][NT][4];
+#pragma unroll
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+      accf[a][nt][0] = accf[a][nt][1] = accf[a][nt][2] = accf[a][nt][3] = 0.f;
+  int ppr = pfirst, pc = i0 - pfirst * nc;         // position of the next item to process
+  bool phasB = ra + ppr * 32 + 16 < rb;
+  const uint2* fb = sfr + lane;
+  auto park = [&]() {
+    float* sp = slots + ((size_t)(warp * g8::kMaxPairsPerWarp + (ppr - pfirst)) * 2 * 32 + lane) * 4 * NT;
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        *reinterpret_cast<float4*>(sp + a * 32 * 4 * NT + nt * 4) =
+            make_float4(accf[a][nt][0], accf[a][nt][1], accf[a][nt][2], accf[a][nt][3]);
+        accf[a][nt][0] = accf[a][nt][1] = accf[a][nt][2] = accf[a][nt][3] = 0.f;
+      }
+  };
+  auto process = [&](const uint4 (&u)[4]) {
+    const uint2* fc = fb + (size_t)pc * 512;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      int ac[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const uint32_t a0 = j ? u[0].z : u[0].x, a2 = j ? u[0].w : u[0].y;
+        const uint32_t a1 = j ? u[1].z : u[1].x, a3 = j ? u[1].w : u[1].y;
+        const uint32_t b0 = j ? u[2].z : u[2].x, b2 = j ? u[2].w : u[2].y;
+        const uint32_t b1 = j ? u[3].z : u[3].x, b3 = j ? u[3].w : u[3].y;
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+          const uint32_t msk = 0x01010101u << p;
+          const uint2 bv = fc[((size_t)nt * P.sc * 16 + j * 8 + p) * 32];
+          imma_u8s8(ac[0], a0 & msk, a1 & msk, a2 & msk, a3 & msk, bv.x, bv.y);
+          if (phasB) imma_u8s8(ac[1], b0 & msk, b1 & msk, b2 & msk, b3 & msk, bv.x, bv.y);
+        }
+      }
+      const float2 w = *reinterpret_cast<const float2*>(wts + (pc * NT + nt) * 8 + 2 * t);
+#pragma unroll
+      for (int a = 0; a < 2; ++a) {
+        accf[a][nt][0] = fmaf((float)ac[a][0], w.x, accf[a][nt][0]);
+        accf[a][nt][1] = fmaf((float)ac[a][1], w.y, accf[a][nt][1]);
+        accf[a][nt][2] = fmaf((float)ac[a][2], w.x, accf[a][nt][2]);
+        accf[a][nt][3] = fmaf((float)ac[a][3], w.y, accf[a][nt][3]);
+      }
+    }
+    // end of this pair's chunks: park the pair's partial in the warp's slot
+    if (++pc == nc) {
+      pc = 0;
+      park();
+      ++ppr;
+      phasB = ra + ppr * 32 + 16 < rb;
+    }
+  };
+
+  for (int kb = 0; kb < n; kb += g8::kPrefetch) {
+#pragma unroll
+    for (int k = 0; k < g8::kPrefetch; ++k) {
+      if (kb + k < n) {
+        process(q[k]);
+        if (kb + k + g8::kPrefetch < n) load_next(q[k]);
+      }
+    }
+  }
+  if (n > 0 && pc != 0) park();   // the run ended inside a pair
+  __syncthreads();
+
+  // ---- 4. per (row, token): this slice's value = its sum of z + warps' partials in warp order
+  const int rows = rb - ra;
+  for (int e = tid; e < rows * P.batch; e += g8::kThreads) {
+    const int tok = e / rows;
+    const int rr = e - tok * rows;
+    const int pr = rr >> 5, a = (rr >> 4) & 1, r = rr & 15;
+    const int nt = tok >> 1, cb = (tok & 1) * 4;
+    // warp w owns items [floor(w*items/16), floor((w+1)*items/16)); item i belongs to warp
+    // ceil(16*(i+1)/items) - 1
+    const int wlo = (int)(((int64_t)(pr * nc + 1) * g8::kWarps + items - 1) / items) - 1;
+    const int whi = (int)(((int64_t)((pr + 1) * nc) * g8::kWarps + items - 1) / items) - 1;
+    float v = 0.f;
+    for (int w = max(0, wlo); w <= min(g8::kWarps - 1, whi); ++w) {
+      const int wi0 = (int)((int64_t)w * items / g8::kWarps);
+      const int wi1 = (int)((int64_t)(w + 1) * items / g8::kWarps);
+      if (wi0 == wi1 || wi1 <= pr * nc || wi0 >= (pr + 1) * nc) continue;
+      const float* sp =
+          slots + ((size_t)(w * g8::kMaxPairsPerWarp + (pr - s_pfirst[w])) * 2 + a) * 32 * 4 * NT;
+#pragma unroll
+      for (int pl = 0; pl < 4; ++pl) {
+        const int col = cb + pl;
+        const int ln = 4 * (r & 7) + (col >> 1);
+        const int i = 2 * (r >> 3) + (col & 1);
+        v += sp[ln * 4 * NT + nt * 4 + i];
+      }
+    }
+    const int row = ra + rr;
+    const float part = s_sumz[tok] + v;
+    if (P.S == 1)
+      P.y[(int64_t)tok * P.N + row] = load_as_f32(P.s, P.sdt, row) * part;
+    else
+      P.partials[((int64_t)sl * P.batch + tok) * P.N + row] = part;
+  }
+  if (P.S == 1) return;
+
+  // ---- cross-slice completion by the last CTA of this row range
+  __threadfence();
+  __syncthreads();
+  uint32_t* ctr = P.counters + ri;
+  if (tid == 0) s_last = (atomicAdd(ctr, 1u) == (uint32_t)(P.S - 1));
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int e = tid; e < rows * P.batch; e += g8::kThreads) {
+    const int tok = e / rows;
+    const int row = ra + (e - tok * rows);
+    float a = 0.f;
+    for (int k = 0; k < P.S; ++k) a += __ldcg(&P.partials[((int64_t)k * P.batch + tok) * P.N + row]);
+    P.y[(int64_t)tok * P.N + row] = load_as_f32(P.s, P.sdt, row) * a;
+  }
+  if (tid == 0) *ctr = 0u;   // ready for the next call on this workspace
+}
+
+// ------------------------------------------------------------------ host side
+
+static int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 0;
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
+static size_t g8_smem(int nt, int sc, int batch, int xs_floats) {
+  return (size_t)nt * sc * g8::kFragBytesPerChunk +
+         (size_t)g8::kWarps * g8::kMaxPairsPerWarp * g8::kSlotFloatsPerNT * nt * 4 +
+         (size_t)batch * xs_floats * 4 + (size_t)g8::kMaxTokens * 128 * 4 +
+         (size_t)sc * nt * 8 * 4 + (size_t)sc * batch * 4;
+}
+
+static int xs_floats_for(int sc, int d, int D, int Bh) {
+  const int span = (sc * 512 / D + 2) * d;
+  return Bh > 0 ? ((span + Bh - 1) / Bh + 1) * Bh : span;
+}
+
+G8Plan plan_gemv_i8(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, int32_t D,
+                    int32_t Bh) {
+  (void)K;
+  G8Plan p{};
+  p.ok = batch >= 1 && batch <= g8::kMaxTokens && L <= (int64_t)1 << 30 && d * D <= 1024;
+  if (!p.ok) return p;
+  const int ntok = (batch + 1) / 2;
+  p.nt = ntok <= 1 ? 1 : ntok <= 2 ? 2 : 4;
+  p.nchunk = (int)((L + 511) / 512);
+  const int sms = sm_count();
+  // about 10 chunks per slice for one token; fewer when the fragments of several tokens or a
+  // large whitening block make the shared memory tight
+  int sc = std::max(1, 10 / p.nt);
+  while (sc > 1 && g8_smem(p.nt, sc, batch, xs_floats_for(sc, d, D, Bh)) > 200 * 1024) --sc;
+  p.S = (p.nchunk + sc - 1) / sc;
+  p.sc = (p.nchunk + p.S - 1) / p.S;
+  p.xs_floats = xs_floats_for(p.sc, d, D, Bh);
+  p.R = std::max(1, std::min(sms / std::min(p.S, sms), (N + 31) / 32));
+  p.nctas = p.S * p.R;
+  // a warp's run must touch at most kMaxPairsPerWarp pairs: ceil(npair/16) + 1 <= 3
+  const int npair = ((N + p.R - 1) / p.R + 31) / 32;
+  if ((npair + g8::kWarps - 1) / g8::kWarps + 1 > g8::kMaxPairsPerWarp) p.ok = false;
+  p.smem = g8_smem(p.nt, p.sc, batch, p.xs_floats);
+  p.ok = p.ok && p.smem <= 220 * 1024;
+  return p;
+}
+
+template <int NT>
+static cudaError_t launch_nt(const G8Plan& pl, const G8Params& P, cudaStream_t st) {
+  static int smem_set[64];
+  cudaError_t e = ensure_smem((const void*)gemv_i8_kernel<NT>, pl.smem, smem_set);
+  if (e != cudaSuccess) return e;
+  gemv_i8_kernel<NT><<<pl.nctas, g8::kThreads, pl.smem, st>>>(P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemv_i8(const G8Plan& pl, const void* x, int xdt, int32_t batch, int32_t K,
+                           Whiten T, const float* M, int32_t d, int32_t D, int64_t L,
+                           const uint32_t* packed, int64_t row_bytes, int32_t N, const void* s,
+                           int sdt, float* y, float* partials, uint32_t* counters,
+                           cudaStream_t st) {
+  G8Params P{};
+  P.x = x;
+  P.xdt = xdt;
+  P.batch = batch;
+  P.K = K;
+  P.T = T;
+  P.M = M;
+  P.d = d;
+  P.D = D;
+  P.L = L;
+  P.packed = reinterpret_cast<const uint8_t*>(packed);
+  P.row_bytes = row_bytes;
+  P.N = N;
+  P.s = s;
+  P.sdt = sdt;
+  P.y = y;
+  P.partials = partials;
+  P.counters = counters;
+  P.nchunk = pl.nchunk;
+  P.sc = pl.sc;
+  P.S = pl.S;
+  P.R = pl.R;
+  P.xs_floats = pl.xs_floats;
+  switch (pl.nt) {
+    case 1: return launch_nt<1>(pl, P, st);
+    case 2: return launch_nt<2>(pl, P, st);
+    default: return launch_nt<4>(pl, P, st);
+  }
+}
+
+}  // namespace lq

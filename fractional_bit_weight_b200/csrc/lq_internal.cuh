@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "liblq.h"
 
 namespace lq {
@@ -30,6 +32,10 @@ __device__ __forceinline__ float load_as_f32(const void* p, int dt, int64_t i) {
   if (dt == LQ_F16) return __half2float(static_cast<const __half*>(p)[i]);
   return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
 }
+
+// Raises the dynamic shared memory limit of `func` to `bytes` on the current device, once per
+// (function, device) and only when a launch needs more than before (keeps launches capturable).
+cudaError_t ensure_smem(const void* func, size_t bytes, int* cache_per_device);
 
 // ---- launchers (host side); each returns cudaGetLastError() of its launch
 cudaError_t launch_pack(const int8_t* b, int32_t N, int64_t L, int64_t words, uint32_t* packed,
@@ -59,5 +65,26 @@ cudaError_t launch_gemv(const GemvPlan& p, const float* z, int64_t L, int32_t ba
                         const uint32_t* packed, int64_t row_words, int32_t N, const void* s,
                         int sdt, float* y, float* partials, uint32_t* counters,
                         cudaStream_t st);
+
+// Plan of the int8 tensor-core GEMV (batch <= 8): S K-slices x R row ranges, one CTA each.
+struct G8Plan {
+  bool ok;
+  int nt;          // 8-column MMA tiles (2 tokens each)
+  int nchunk;      // 512-bit chunks per row
+  int sc;          // chunks per slice
+  int S;           // slices
+  int R;           // row ranges
+  int nctas;       // S * R
+  int xs_floats;   // whitening scratch per token
+  size_t smem;     // dynamic shared memory per CTA
+};
+G8Plan plan_gemv_i8(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, int32_t D,
+                    int32_t Bh);
+// partials: [S][batch][N] floats and counters: [R] zeroed uint32 (both unused when S == 1)
+cudaError_t launch_gemv_i8(const G8Plan& pl, const void* x, int xdt, int32_t batch, int32_t K,
+                           Whiten T, const float* M, int32_t d, int32_t D, int64_t L,
+                           const uint32_t* packed, int64_t row_bytes, int32_t N, const void* s,
+                           int sdt, float* y, float* partials, uint32_t* counters,
+                           cudaStream_t st);
 
 }  // namespace lq

@@ -6,42 +6,9 @@
 // transform (log2 Bh butterfly stages) in shared memory.
 // Lift (paper sec. 3 intro: o = diag(s) W (M T a); review: T* = lift o T):
 // z[g*D + j] = sum_{i<d} M[i][j] xt[g*d + i], xt zero beyond K.
-#include "lq_internal.cuh"
+#include "lq_device.cuh"
 
 namespace lq {
-
-// Whitens Hadamard blocks [blk0, blk0 + nblk) of one input row into sm[0 .. nblk*Bh).
-// All threads of the CTA take part; ends with a barrier.
-__device__ void whiten_blocks_smem(const void* __restrict__ x, int xdt, int64_t row_off, int K,
-                                   const Whiten& T, int blk0, int nblk, float* sm) {
-  const int Bh = T.block;
-  const int n = nblk * Bh;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const int k = blk0 * Bh + i;
-    float v = 0.f;
-    if (k < K) {
-      v = load_as_f32(x, xdt, row_off + k);
-      if (T.chan_scale) v *= T.chan_scale[k];
-      if (T.sign && T.sign[k] < 0) v = -v;
-    }
-    sm[i] = v;
-  }
-  __syncthreads();
-  for (int h = 1; h < Bh; h <<= 1) {
-    for (int p = threadIdx.x; p < n / 2; p += blockDim.x) {
-      const int lo = p & (h - 1);
-      const int i = ((p - lo) << 1) | lo;  // bit h of i is clear; partner is i + h
-      const float a = sm[i], b = sm[i + h];
-      sm[i] = a + b;
-      sm[i + h] = a - b;
-    }
-    __syncthreads();
-  }
-  if (T.inv_sqrt != 1.f) {
-    for (int i = threadIdx.x; i < n; i += blockDim.x) sm[i] *= T.inv_sqrt;
-    __syncthreads();
-  }
-}
 
 // One CTA per (Hadamard block, token).
 __global__ void whiten_kernel(const void* __restrict__ x, int xdt, int K, Whiten T,
@@ -106,6 +73,18 @@ __global__ void lift_f32_kernel(const void* __restrict__ x, int xdt, int K, Whit
   }
 }
 
+cudaError_t ensure_smem(const void* func, size_t bytes, int* cache_per_device) {
+  if (bytes == 0) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cache_per_device[dev] >= (int)bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) cache_per_device[dev] = (int)bytes;
+  return e;
+}
+
 cudaError_t launch_whiten(const void* x, int xdt, int32_t batch, int32_t K, Whiten T,
                           float* xt, cudaStream_t st) {
   if (batch == 0) return cudaSuccess;
@@ -132,12 +111,9 @@ cudaError_t launch_lift_f32(const void* x, int xdt, int32_t batch, int32_t K, Wh
   else
     sx_floats = span;
   const size_t smem = (size_t)(LQ_MAX_D * LQ_MAX_D + sx_floats) * sizeof(float);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(lift_f32_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-  }
+  static int smem_set[64];
+  cudaError_t e = ensure_smem((const void*)lift_f32_kernel, smem, smem_set);
+  if (e != cudaSuccess) return e;
   dim3 grid((G + gpc - 1) / gpc, batch);
   lift_f32_kernel<<<grid, 256, smem, st>>>(x, xdt, K, T, M, d, D, G, gpc, z, zero_ptr,
                                            zero_words);
