@@ -13,8 +13,11 @@ import torch
 
 __all__ = [
     "LQError", "lib", "abi_version", "lifted_bits", "row_stride_bytes", "pack", "unpack",
-    "whiten", "lift", "gemm_workspace_bytes", "gemm", "new_workspace", "device_status",
+    "whiten", "lift", "gemm_workspace_bytes", "gemm", "gemm_noalloc", "new_workspace",
+    "device_status", "NOALLOC_SCRATCH_BYTES",
 ]
+
+NOALLOC_SCRATCH_BYTES = 8 << 20   # LQ_NOALLOC_SCRATCH_BYTES
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "liblq.so")
@@ -24,8 +27,8 @@ LQ_F32, LQ_F16, LQ_BF16 = 0, 1, 2
 _DTYPES = {torch.float32: LQ_F32, torch.float16: LQ_F16, torch.bfloat16: LQ_BF16}
 
 EXPORTS = ("lq_abi_version", "lq_lifted_bits", "lq_row_stride_bytes", "lq_pack", "lq_unpack",
-           "lq_whiten", "lq_lift", "lq_gemm_workspace_bytes", "lq_gemm", "lq_device_status",
-           "lq_status_string", "lq_last_error")
+           "lq_whiten", "lq_lift", "lq_gemm_workspace_bytes", "lq_gemm", "lq_gemm_noalloc",
+           "lq_device_status", "lq_status_string", "lq_last_error")
 
 
 class LQError(RuntimeError):
@@ -56,6 +59,8 @@ def _declare(L):
         "lq_gemm_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
         "lq_gemm": ([vp, ctypes.c_int, i32, dp, vp, vp, vp, ctypes.c_int, i32, i32, i32, i32, vp,
                      vp, sz, vp], ctypes.c_int),
+        "lq_gemm_noalloc": ([vp, ctypes.c_int, i32, dp, vp, vp, vp, ctypes.c_int, i32, i32, i32,
+                             i32, vp, vp], ctypes.c_int),
         "lq_device_status": ([vp, ctypes.POINTER(i32), vp], ctypes.c_int),
         "lq_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "lq_last_error": ([], ctypes.c_char_p),
@@ -197,6 +202,27 @@ def gemm(x, packed, M, s, d, D, sign=None, chan_scale=None, block=0, y=None, wor
                          _dev(y, "y", (torch.float32,)), _dev(workspace, "workspace"),
                          workspace.numel() * workspace.element_size(), _stream(stream)),
            "lq_gemm")
+    return y
+
+
+def gemm_noalloc(x, packed, M, s, d, D, sign=None, chan_scale=None, block=0, y=None,
+                 stream=None):
+    """lq_gemm without a workspace: the library's own fixed device scratch is used (batch 1..8).
+
+    For callers that cannot allocate device memory. The first call on a device sets it up and
+    should come before any stream capture; calls that overlap on the GPU share the scratch and
+    must be serialised by the caller.
+    """
+    batch, K = x.shape
+    N = packed.shape[0]
+    if y is None:
+        y = torch.empty((batch, N), dtype=torch.float32, device=x.device)
+    desc = _whiten_desc(sign, chan_scale, block)
+    _check(lib().lq_gemm_noalloc(_dev(x, "x", _DTYPES), _DTYPES[x.dtype], batch, _desc_ptr(desc),
+                                 _dev(packed, "packed", (torch.int32,)),
+                                 _dev(M, "M", (torch.float32,)), _dev(s, "s", _DTYPES),
+                                 _DTYPES[s.dtype], d, D, K, N, _dev(y, "y", (torch.float32,)),
+                                 _stream(stream)), "lq_gemm_noalloc")
     return y
 
 

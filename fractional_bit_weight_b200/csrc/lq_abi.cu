@@ -110,6 +110,21 @@ constexpr int32_t kMaxK = 1 << 24;
 
 }  // namespace
 
+namespace lq {
+
+void set_last_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+}
+
+lq_status whiten_from_desc(const lq_whiten_desc* T, int32_t K, Whiten* out) {
+  return make_whiten(T, K, out);
+}
+
+}  // namespace lq
+
 extern "C" {
 
 int32_t lq_abi_version(void) { return LQ_ABI_VERSION; }

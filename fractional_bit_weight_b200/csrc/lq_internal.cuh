@@ -33,6 +33,11 @@ __device__ __forceinline__ float load_as_f32(const void* p, int dt, int64_t i) {
   return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
 }
 
+// Records the reason for a rejected call (read back by lq_last_error on this host thread).
+void set_last_error(const char* fmt, ...);
+// Validates a whitening descriptor against K (as lq_gemm does) and converts it.
+lq_status whiten_from_desc(const lq_whiten_desc* T, int32_t K, Whiten* out);
+
 // Raises the dynamic shared memory limit of `func` to `bytes` on the current device, once per
 // (function, device) and only when a launch needs more than before (keeps launches capturable).
 cudaError_t ensure_smem(const void* func, size_t bytes, int* cache_per_device);

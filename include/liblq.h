@@ -131,6 +131,32 @@ LQ_API lq_status lq_gemm(const void* x, lq_dtype xdt, int32_t batch, const lq_wh
                   int32_t d, int32_t D, int32_t K, int32_t N, float* y, void* workspace,
                   size_t workspace_bytes, lq_stream stream);
 
+/* Bytes of the scratch array that lq_gemm_noalloc keeps on every device that loads the library. */
+#define LQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* lq_gemm for callers that cannot allocate device memory. The paper has no counterpart: this is
+ * a deployment entry point of this library, not a step of the method.
+ * Some callers cannot hand the library a workspace: their device memory is owned by a host
+ * framework or allocator they cannot call into (a plugin, an inference-server backend with a
+ * fixed budget), or they run where allocating is not allowed. This entry point takes the same
+ * arguments as lq_gemm except the workspace, allocates nothing (no cudaMalloc, no cudaFree, no
+ * allocating library routine) and keeps its scratch (split-K counters and slice partials) in a
+ * fixed device array of LQ_NOALLOC_SCRATCH_BYTES bytes that every GPU which loads the library
+ * holds until the process exits.
+ *   - batch 1..8 (the small-batch GEMV); shapes whose scratch would exceed
+ *     LQ_NOALLOC_SCRATCH_BYTES are rejected with LQ_EINVAL and a reason in lq_last_error().
+ *   - The first call on a device sets that device up (finds the array's device address and
+ *     clears its counters, synchronising the device): make that first call before any stream
+ *     capture.
+ *   - Every call on a device shares the one array and leaves it ready for the next call; calls
+ *     that overlap on the GPU (different streams, or threads without ordering) race on it and
+ *     must be serialised by the caller.
+ * Errors: as lq_gemm, plus LQ_EINVAL for batch > 8 or a scratch need above the maximum. */
+LQ_API lq_status lq_gemm_noalloc(const void* x, lq_dtype xdt, int32_t batch,
+                                 const lq_whiten_desc* T, const uint32_t* packed, const float* M,
+                                 const void* s, lq_dtype sdt, int32_t d, int32_t D, int32_t K,
+                                 int32_t N, float* y, lq_stream stream);
+
 /* Synchronise `stream`, then read the workspace status word into *code (0 = no device-side
  * failure) and clear it. Returns LQ_OK, or the lq_status that the word records. */
 LQ_API lq_status lq_device_status(void* workspace, int32_t* code, lq_stream stream);
