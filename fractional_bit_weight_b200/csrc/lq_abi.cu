@@ -72,7 +72,7 @@ lq_status make_whiten(const lq_whiten_desc* T, int32_t K, lq::Whiten* out) {
 struct WsLayout {
   int path;          // 0: int8 tensor-core GEMV (batch <= 8); 1: fp32 GEMV over z
   size_t counters;   // uint32 completion counters of the split-K reduction
-  size_t z;          // float z [batch][L] (path 1)
+  size_t z;          // path 0: prep output (fragments, weights, sums); path 1: float z [batch][L]
   size_t partials;   // float [slices][batch][N]
   size_t total;
   lq::GemvPlan gemv;
@@ -88,6 +88,7 @@ WsLayout layout_gemm(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D, 
   if (w.path == 0) {
     ncounters = (size_t)w.g8.R;
     npartials = w.g8.S > 1 ? (size_t)w.g8.S * batch * N : 0;
+    nz = (w.g8.frag_bytes + w.g8.wtab_bytes + w.g8.csum_bytes + 3) / 4;   // prep output
   } else {
     w.gemv = lq::plan_gemv(batch, L, N);
     ncounters = (size_t)w.gemv.ntg * w.gemv.ntiles;
@@ -252,8 +253,8 @@ lq_status lq_gemm(const void* x, lq_dtype xdt, int32_t batch, const lq_whiten_de
   float* partials = reinterpret_cast<float*>(ws + lay.partials);
   if (lay.path == 0) {
     cudaError_t e = lq::launch_gemv_i8(lay.g8, x, (int)xdt, batch, K, w, M, d, D, L, packed,
-                                       row_stride_bytes(K, d, D), N, s, (int)sdt, y, partials,
-                                       counters, cs);
+                                       row_stride_bytes(K, d, D), N, s, (int)sdt, y, ws + lay.z,
+                                       partials, counters, cs);
     return e == cudaSuccess ? LQ_OK : cuda_fail(e, "lq_gemm (int8 gemv)");
   }
   if (lay.gemv.ntiles > 65535 || lay.gemv.ntg > 65535)

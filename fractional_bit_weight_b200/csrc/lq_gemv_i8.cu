@@ -1,4 +1,4 @@
-// lq_gemv_i8.cu -- decode GEMV for small batches (batch <= 8), one kernel per call.
+// lq_gemv_i8.cu -- decode GEMV for small batches (batch <= 8).
 //
 // y[t][n] = s[n] * sum_q b[n][q] z[t][q] with b in {+1,-1}, z = lift(T(x[t]))
 // (paper sec. 3 intro: o = diag(s) W (M T a); review "Method": an INT1 x FP product plus small
@@ -6,26 +6,24 @@
 //     sum_q b_q z_q = sum_q z_q - 2 * sum_{q: bit_q = 1} z_q,
 // so each row needs only the subset sum of z over its set bits.
 //
-// The lifted dimension is cut into 512-bit chunks and the chunks into S slices; the grid is
-// S slices x R row ranges, one CTA each (one CTA per SM). A CTA:
-//  1. starts streaming its first stored bits into registers;
-//  2. prologue, in shared memory: whitens the Hadamard blocks that feed its slice (one warp per
-//     block: the first butterfly stages in registers, the rest with lane shuffles), lifts them,
-//     z = M^T xt per block of d inputs (one value per thread at a time), picks a power-of-two
-//     scale S from max|z| of each chunk, and splits z*S*2^-p, p = q mod 8, into four int8
-//     planes (base 254) written in the register layout of the B operand of mma.m16n8k32
-//     (8 columns = 2 tokens x 4 planes), with the chunk's column weights -2*254^-plane/S and
-//     its sum of z;
-//  3. main loop: the (32-row tile pair, chunk) items of its rows, pair-major, in 16 equal
-//     contiguous runs, one per warp. A 32-bit word of stored bits becomes an int8 A operand
-//     with one AND, (w & 0x01010101 << p): bit p of each byte as 0 or 2^p; the B entries carry
-//     2^-p, so all eight bit positions accumulate into one int32 set per item, scaled to fp32
-//     by the chunk's column weights;
-//  4. warps park the fp32 partial of every pair they touched in their own shared-memory slot;
-//     the slots are summed in warp order. With S > 1 each CTA writes its slice's partial and
-//     the last CTA of a row range to finish adds the slices in slice order and applies s.
-// Every CTA of a slice computes identical fragments, and all sums run in a fixed order, so the
-// result does not depend on timing.
+// Two kernels per call, the second launched with programmatic dependent launch:
+//  prep, one CTA per 512-bit chunk of the lifted dimension: whitens the Hadamard blocks that
+//    feed the chunk (a warp per block: the first butterfly stages in registers, the rest with
+//    lane shuffles), lifts them, z = M^T xt per block of d inputs, picks a power-of-two scale S
+//    from max|z| of the chunk, and splits z*S*2^-p, p = q mod 8, into four int8 planes (base
+//    254) stored in the register layout of the B operand of mma.m16n8k32 (8 columns = 2 tokens
+//    x 4 planes), with the chunk's column weights -2*254^-plane/S and its sum of z.
+//  gemv, S slices of chunks x R row ranges, one CTA each (one per SM): starts streaming its
+//    stored bits into registers at once, waits for prep, copies its slice's fragments to shared
+//    memory, then runs the (32-row tile pair, chunk) items of its rows, pair-major, in 16 equal
+//    contiguous runs, one per warp. A 32-bit word of stored bits becomes an int8 A operand with
+//    one AND, (w & 0x01010101 << p): bit p of each byte as 0 or 2^p; the B entries carry 2^-p,
+//    so all eight bit positions accumulate into one int32 set per item, which the chunk's column
+//    weights turn into fp32. Warps park the fp32 partial of every pair they touched in their own
+//    shared-memory slot, summed in warp order at the end; with S > 1 the last CTA of a row range
+//    to finish adds the slices in slice order and applies s.
+// Fragments are computed once per call and every sum runs in a fixed order, so the result does
+// not depend on timing.
 #include "lq_device.cuh"
 
 namespace lq {
@@ -40,7 +38,7 @@ constexpr int kMaxPairsPerWarp = 3;               // fp32 partial slots per warp
 constexpr int kSlotFloatsPerNT = 2 * 32 * 4;      // one tile pair: 2 tiles x 32 lanes x 4 regs
 }  // namespace g8
 
-struct G8Params {
+struct PrepParams {
   const void* x;
   int xdt;
   int batch;
@@ -50,19 +48,31 @@ struct G8Params {
   int d;
   int D;
   int64_t L;
+  int nchunk;
+  int sc;               // chunks per slice (fragments are stored slice by slice)
+  int xs_floats;        // whitening scratch per token
+  uint2* frags;         // [S][NT][sc][16][32]
+  float* wtab;          // [nchunk][NT][8]
+  float* csum;          // [nchunk][batch]
+};
+
+struct G8Params {
   const uint8_t* packed;
   int64_t row_bytes;
   int N;
   const void* s;
   int sdt;
   float* y;
+  int batch;
+  const uint2* frags;
+  const float* wtab;
+  const float* csum;
   float* partials;      // [S][batch][N] when S > 1
   uint32_t* counters;   // [R] when S > 1
   int nchunk;           // 512-bit chunks per row
   int sc;               // chunks per slice
   int S;                // slices
   int R;                // row ranges
-  int xs_floats;        // whitening scratch per token
 };
 
 __device__ __forceinline__ void imma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -105,75 +115,26 @@ __device__ __forceinline__ void planes4(float a, int (&P)[4]) {
   P[3] = __float2int_rn(r);
 }
 
+constexpr int kPrepThreads = 512;
+
+// One CTA per chunk; see the file comment.
 template <int NT>
-__global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params P) {
+__global__ void __launch_bounds__(kPrepThreads) gemv_i8_prep_kernel(const PrepParams P) {
+  // let the dependent gemv grid launch now; it waits for this grid before reading our output
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ __align__(16) uint8_t smem[];
-  __shared__ float s_sumz[g8::kMaxTokens];
-  __shared__ float s_scale[16 * g8::kMaxTokens];   // per (chunk, token); chunks per slice <= 16
-  __shared__ int s_pfirst[g8::kWarps];
-  __shared__ int s_last;
+  __shared__ float s_red[2][g8::kMaxTokens][kPrepThreads / 32];
+  __shared__ float s_scale[g8::kMaxTokens];
+  float* xs = reinterpret_cast<float*>(smem);                       // [batch][xs_floats]
+  float* zs = xs + (size_t)P.batch * P.xs_floats;                   // [batch][512 + pad]
+  float* Ms = zs + (size_t)P.batch * 576;                           // [d][D]
+  constexpr int kZP = 576;   // 512 values + 8 pad floats per 128 (bank-conflict-free reads)
 
+  const int c = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int sl = blockIdx.x % P.S, ri = blockIdx.x / P.S;
-  const int c0 = sl * P.sc;
-  const int nc = min(P.sc, P.nchunk - c0);
-  const int ra = (int)((int64_t)ri * P.N / P.R);
-  const int rb = (int)((int64_t)(ri + 1) * P.N / P.R);
-  const int npair = (rb - ra + 31) / 32;
-  const int items = npair * nc;
-  const int i0 = (int)((int64_t)warp * items / g8::kWarps);
-  const int i1 = (int)((int64_t)(warp + 1) * items / g8::kWarps);
-  const int n = i1 - i0;
-  const int pfirst = i0 / nc;
-
-  constexpr int kSlotFloats = g8::kSlotFloatsPerNT * NT;
-  uint2* sfr = reinterpret_cast<uint2*>(smem);                                  // [NT][sc][16][32]
-  float* slots = reinterpret_cast<float*>(smem + (size_t)NT * P.sc * g8::kFragBytesPerChunk);
-  float* xs = slots + (size_t)g8::kWarps * g8::kMaxPairsPerWarp * kSlotFloats;  // [batch][xs_floats]
-  float* Ms = xs + (size_t)P.batch * P.xs_floats;                               // [d][D]
-  float* wts = Ms + g8::kMaxTokens * 128;                                       // [sc][NT][8]
-  float* csum = wts + (size_t)P.sc * NT * 8;                                    // [sc][batch]
-
-  // ---- 1. start streaming: item i = (pair i / nc, chunk c0 + i % nc)
-  const int64_t last_off = P.row_bytes - 16;
-  int lpr = pfirst, lc = i0 - pfirst * nc;       // position of the next item to load
-  const uint8_t* rowp[4];
-  bool lhasB = false;
-  auto set_rows = [&](int pr) {
-    const int r = ra + pr * 32 + g;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int row = r + 8 * k;
-      rowp[k] = P.packed + (int64_t)(row < rb ? row : ra) * P.row_bytes + 16 * t;
-    }
-    lhasB = ra + pr * 32 + 16 < rb;
-  };
-  auto load_next = [&](uint4 (&u)[4]) {
-    int64_t off = (int64_t)(c0 + lc) * 64;
-    off = off + 16 * t > last_off ? last_off - 16 * t : off;   // last chunk: stay in the row
-    u[0] = ldg_stream_v4(rowp[0] + off);
-    u[1] = ldg_stream_v4(rowp[1] + off);
-    if (lhasB) {
-      u[2] = ldg_stream_v4(rowp[2] + off);
-      u[3] = ldg_stream_v4(rowp[3] + off);
-    }
-    if (++lc == nc) {
-      lc = 0;
-      if (++lpr < npair) set_rows(lpr);
-    }
-  };
-  if (n > 0) set_rows(lpr);
-  uint4 q[g8::kPrefetch][4];
-#pragma unroll
-  for (int k = 0; k < g8::kPrefetch; ++k)
-    if (k < n) load_next(q[k]);
-
-  // ---- 2. prologue: this slice's fragments, column weights and chunk sums
-  if (lane == 0) s_pfirst[warp] = pfirst;
-  for (int i = tid; i < P.d * P.D; i += g8::kThreads) Ms[i] = P.M[i];
-  const int64_t q0 = (int64_t)c0 * 512;
-  const int64_t q1 = min((int64_t)(c0 + nc) * 512, P.L);
+  const int64_t q0 = (int64_t)c * 512;
+  const int64_t q1 = min(q0 + 512, P.L);
+  const int nq = (int)(q1 - q0);
   const int g_lo = (int)(q0 / P.D), g_hi = (int)((q1 - 1) / P.D);
   const int k0 = g_lo * P.d;
   const int k1 = min((g_hi + 1) * P.d, P.K);
@@ -184,11 +145,12 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
     base = blk0 * Bh;
     span = ((k1 + Bh - 1) / Bh - blk0) * Bh;
   }
+  for (int i = tid; i < P.d * P.D; i += kPrepThreads) Ms[i] = P.M[i];
+  // 1. whitened inputs of every token
   if (Bh >= 32 && Bh <= 256) {
-    // one warp per (token, block); lane l holds elements [E*l, E*l + E)
     const int E = Bh >> 5;
     const int nblk = span / Bh;
-    for (int task = warp; task < P.batch * nblk; task += g8::kWarps) {
+    for (int task = warp; task < P.batch * nblk; task += kPrepThreads / 32) {
       const int tok = task / nblk, b = task - tok * nblk;
       float v[8];
 #pragma unroll
@@ -228,7 +190,7 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
     }
     __syncthreads();
   } else {
-    for (int e = tid; e < P.batch * span; e += g8::kThreads) {
+    for (int e = tid; e < P.batch * span; e += kPrepThreads) {
       const int tok = e / span, i = e - tok * span;
       const int k = base + i;
       float a = 0.f;
@@ -245,7 +207,7 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
     if (Bh > 1) {
       const int half = span / 2;
       for (int h = 1; h < Bh; h <<= 1) {
-        for (int pp = tid; pp < P.batch * half; pp += g8::kThreads) {
+        for (int pp = tid; pp < P.batch * half; pp += kPrepThreads) {
           const int tok = pp / half, pi = pp - tok * half;
           const int lo = pi & (h - 1);
           const int i = ((pi - lo) << 1) | lo;
@@ -258,73 +220,69 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
       }
     }
   }
-  // lift: every thread computes whole values z[e] of the slice (e = 512 * chunk + offset),
-  // all tokens, into shared memory (the lift runs over the d inputs of the value's block)
-  float* zs = slots;   // the partial slots are free until the main loop
-  const int nq = (int)(q1 - q0);
-  for (int tok = 0; tok < P.batch; ++tok) {
-    const float* xt = xs + tok * P.xs_floats;
-    for (int e = tid; e < nc * 512; e += g8::kThreads) {
+  // 2. lift: thread tid owns value e = tid of every token; per-warp max and sum
+  {
+    const int e = tid;
+    int gg = 0, jj = 0, dv = 0;
+    if (e < nq) {
+      const int qi = (int)(q0 + e);
+      gg = qi / P.D;
+      jj = qi - gg * P.D;
+      dv = min(P.d, P.K - gg * P.d);
+    }
+    for (int tok = 0; tok < P.batch; ++tok) {
       float acc = 0.f;
-      if (e < nq) {
-        const int qi = (int)(q0 + e);
-        const int gg = qi / P.D;
-        const int jj = qi - gg * P.D;
-        const float* xg = xt + (gg * P.d - base);
-        const float* mj = Ms + jj;
-        const int dv = min(P.d, P.K - gg * P.d);   // inputs past K are zero
-        for (int ii = 0; ii < dv; ++ii) acc = fmaf(mj[ii * P.D], xg[ii], acc);
-        acc *= P.T.inv_sqrt;
+      const float* xg = xs + tok * P.xs_floats + (gg * P.d - base);
+      for (int ii = 0; ii < dv; ++ii) acc = fmaf(Ms[ii * P.D + jj], xg[ii], acc);
+      acc *= P.T.inv_sqrt;
+      zs[tok * kZP + e + 8 * (e >> 7)] = acc;
+      const float m = warp_max(fabsf(acc));
+      const float su = warp_sum(acc);
+      if (lane == 0) {
+        s_red[0][tok][warp] = m;
+        s_red[1][tok][warp] = su;
       }
-      zs[tok * (P.sc * 512) + e] = acc;
     }
   }
   __syncthreads();
-  // per (chunk, token): max|z| -> power-of-two scale, and the sum of z; one warp each
-  for (int task = warp; task < nc * P.batch; task += g8::kWarps) {
-    const int cl = task / P.batch, tok = task - cl * P.batch;
-    const float* zc = zs + tok * (P.sc * 512) + cl * 512;
-    float lmax = 0.f, lsum = 0.f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float v = zc[lane + 32 * i];
-      lmax = fmaxf(lmax, fabsf(v));
-      lsum += v;
+  if (tid < P.batch) {
+    float m = 0.f, su = 0.f;
+    for (int w = 0; w < kPrepThreads / 32; ++w) {
+      m = fmaxf(m, s_red[0][tid][w]);
+      su += s_red[1][tid][w];
     }
-    const float m = warp_max(lmax);
-    const float su = warp_sum(lsum);
-    if (lane == 0) {
+    int ex = 0;
+    frexpf(m, &ex);                                         // m = f * 2^ex, f in [0.5, 1)
+    const float S = m > 0.f ? ldexpf(1.f, 6 - ex) : 1.f;    // |z| * S < 64
+    s_scale[tid] = S;
+    P.csum[(int64_t)c * P.batch + tid] = su;
+  }
+  if (tid < NT * 8) {
+    const int nt = tid >> 3, col = tid & 7, tok = nt * 2 + (col >> 2), pl = col & 3;
+    float w = 0.f;
+    if (tok < P.batch) {
+      float m = 0.f;
+      for (int ww = 0; ww < kPrepThreads / 32; ++ww) m = fmaxf(m, s_red[0][tok][ww]);
       int ex = 0;
-      frexpf(m, &ex);                                         // m = f * 2^ex, f in [0.5, 1)
-      const float Ssc = m > 0.f ? ldexpf(1.f, 6 - ex) : 1.f;  // |z| * S < 64
-      csum[cl * P.batch + tok] = su;
-      const int nt = tok >> 1, cb = (tok & 1) * 4;
-      float w = -2.f / Ssc;
-      for (int pl = 0; pl < 4; ++pl) {
-        wts[(cl * NT + nt) * 8 + cb + pl] = w;
-        w *= (float)(1.0 / 254.0);
-      }
-      s_scale[cl * g8::kMaxTokens + tok] = Ssc;
+      frexpf(m, &ex);
+      w = -2.f / (m > 0.f ? ldexpf(1.f, 6 - ex) : 1.f);
+      for (int k = 0; k < pl; ++k) w *= (float)(1.0 / 254.0);
     }
-  }
-  // weights of unused token columns
-  for (int i = tid; i < nc * NT * 8; i += g8::kThreads) {
-    const int col = i & 7, nt = (i >> 3) % NT;
-    if (nt * 2 + (col >> 2) >= P.batch) wts[i] = 0.f;
+    P.wtab[(int64_t)c * NT * 8 + tid] = w;
   }
   __syncthreads();
-  // quantise: a group (chunk, token slot, tt, j, h, p) is 4 values e0 + 8*i, i = 0..3, which
-  // fill one 32-bit word per plane: word (j*8 + p)*64 + 2*(4*col + tt) + h of the chunk
-  for (int gi = tid; gi < nc * 2 * NT * 128; gi += g8::kThreads) {
-    const int cl = gi / (2 * NT * 128);
-    const int rem = gi - cl * (2 * NT * 128);
-    const int tok = rem >> 7, grp = rem & 127;
-    const int tt = grp >> 5, jl = (grp >> 4) & 1, hl = (grp >> 3) & 1, pl8 = grp & 7;
+  // 3. quantise and store: thread -> (token slot, tt, j, h, p); its 4 values e0 + 8*i fill one
+  // 32-bit word per plane, word (j*8 + p)*64 + 2*(4*col + tt) + h of the chunk's fragment block
+  const int sl = c / P.sc, cl = c - sl * P.sc;
+  for (int gi = tid; gi < 2 * NT * 128; gi += kPrepThreads) {
+    const int tok = gi >> 7, grp = gi & 127;
+    const int pl8 = grp & 7, tt = (grp >> 3) & 3, hl = (grp >> 5) & 1, jl = grp >> 6;
     const int nt = tok >> 1, cb = (tok & 1) * 4;
     uint32_t w4[4] = {0u, 0u, 0u, 0u};
     if (tok < P.batch) {
-      const float Sp = s_scale[cl * g8::kMaxTokens + tok] * __int_as_float((127 - pl8) << 23);
-      const float* zc = zs + tok * (P.sc * 512) + cl * 512 + 128 * tt + 64 * jl + 32 * hl + pl8;
+      const float Sp = s_scale[tok] * __int_as_float((127 - pl8) << 23);   // S * 2^-p, exact
+      const int e0 = 128 * tt + 64 * jl + 32 * hl + pl8;
+      const float* zc = zs + tok * kZP + e0 + 8 * tt;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         int Pq[4];
@@ -333,16 +291,94 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
         for (int pl = 0; pl < 4; ++pl) w4[pl] |= ((uint32_t)Pq[pl] & 0xffu) << (8 * i);
       }
     }
-    uint32_t* fw = reinterpret_cast<uint32_t*>(sfr) + ((size_t)nt * P.sc + cl) * (g8::kFragBytesPerChunk / 4);
+    uint32_t* fw = reinterpret_cast<uint32_t*>(P.frags) +
+                   (((size_t)sl * NT + nt) * P.sc + cl) * (g8::kFragBytesPerChunk / 4);
 #pragma unroll
     for (int pl = 0; pl < 4; ++pl) fw[(jl * 8 + pl8) * 64 + 2 * (4 * (cb + pl) + tt) + hl] = w4[pl];
   }
-  __syncthreads();
-  if (tid < P.batch) {
-    float a = 0.f;
-    for (int c = 0; c < nc; ++c) a += csum[c * P.batch + tid];
-    s_sumz[tid] = a;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params P) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  __shared__ float s_sumz[g8::kMaxTokens];
+  __shared__ int s_pfirst[g8::kWarps];
+  __shared__ int s_last;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int sl = blockIdx.x % P.S, ri = blockIdx.x / P.S;
+  const int c0 = sl * P.sc;
+  const int nc = min(P.sc, P.nchunk - c0);
+  const int ra = (int)((int64_t)ri * P.N / P.R);
+  const int rb = (int)((int64_t)(ri + 1) * P.N / P.R);
+  const int npair = (rb - ra + 31) / 32;
+  const int items = npair * nc;
+  const int i0 = (int)((int64_t)warp * items / g8::kWarps);
+  const int i1 = (int)((int64_t)(warp + 1) * items / g8::kWarps);
+  const int n = i1 - i0;
+  const int pfirst = i0 / nc;
+
+  constexpr int kSlotFloats = g8::kSlotFloatsPerNT * NT;
+  uint2* sfr = reinterpret_cast<uint2*>(smem);                                  // [NT][sc][16][32]
+  float* slots = reinterpret_cast<float*>(smem + (size_t)NT * P.sc * g8::kFragBytesPerChunk);
+  float* wts = slots + (size_t)g8::kWarps * g8::kMaxPairsPerWarp * kSlotFloats; // [sc][NT][8]
+
+  // ---- 1. start streaming: item i = (pair i / nc, chunk c0 + i % nc)
+  const int64_t last_off = P.row_bytes - 16;
+  int lpr = pfirst, lc = i0 - pfirst * nc;       // position of the next item to load
+  const uint8_t* rowp[4];
+  bool lhasB = false;
+  auto set_rows = [&](int pr) {
+    const int r = ra + pr * 32 + g;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int row = r + 8 * k;
+      rowp[k] = P.packed + (int64_t)(row < rb ? row : ra) * P.row_bytes + 16 * t;
+    }
+    lhasB = ra + pr * 32 + 16 < rb;
+  };
+  auto load_next = [&](uint4 (&u)[4]) {
+    int64_t off = (int64_t)(c0 + lc) * 64;
+    off = off + 16 * t > last_off ? last_off - 16 * t : off;   // last chunk: stay in the row
+    u[0] = ldg_stream_v4(rowp[0] + off);
+    u[1] = ldg_stream_v4(rowp[1] + off);
+    if (lhasB) {
+      u[2] = ldg_stream_v4(rowp[2] + off);
+      u[3] = ldg_stream_v4(rowp[3] + off);
+    }
+    if (++lc == nc) {
+      lc = 0;
+      if (++lpr < npair) set_rows(lpr);
+    }
+  };
+  if (n > 0) set_rows(lpr);
+  uint4 q[g8::kPrefetch][4];
+#pragma unroll
+  for (int k = 0; k < g8::kPrefetch; ++k)
+    if (k < n) load_next(q[k]);
+  if (lane == 0) s_pfirst[warp] = pfirst;
+
+  // ---- 2. this slice's fragments and column weights (written by the prep kernel)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  {
+    const int nvec = NT * P.sc * g8::kFragBytesPerChunk / 16;
+    const uint4* src = reinterpret_cast<const uint4*>(P.frags) + (size_t)sl * nvec;
+    uint4* dst = reinterpret_cast<uint4*>(sfr);
+    for (int i = tid; i < nvec; i += g8::kThreads) {
+      const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst + i);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src + i) : "memory");
+    }
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+    for (int i = tid; i < nc * NT * 8; i += g8::kThreads) wts[i] = P.wtab[(size_t)c0 * NT * 8 + i];
+    if (tid < P.batch) {
+      float a = 0.f;
+      for (int c = 0; c < nc; ++c) a += P.csum[(int64_t)(c0 + c) * P.batch + tid];
+      s_sumz[tid] = a;
+    }
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
   }
+  __syncthreads();
 
   // ---- 3. main loop
   float accf[2][NT][4];
@@ -369,7 +405,11 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
     const uint2* fc = fb + (size_t)pc * 512;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      int ac[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+      int ac[2][2][4];   // [tile][k-half]: four independent accumulation chains
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) ac[a][j][0] = ac[a][j][1] = ac[a][j][2] = ac[a][j][3] = 0;
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const uint32_t a0 = j ? u[0].z : u[0].x, a2 = j ? u[0].w : u[0].y;
@@ -380,17 +420,17 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
         for (int p = 0; p < 8; ++p) {
           const uint32_t msk = 0x01010101u << p;
           const uint2 bv = fc[((size_t)nt * P.sc * 16 + j * 8 + p) * 32];
-          imma_u8s8(ac[0], a0 & msk, a1 & msk, a2 & msk, a3 & msk, bv.x, bv.y);
-          if (phasB) imma_u8s8(ac[1], b0 & msk, b1 & msk, b2 & msk, b3 & msk, bv.x, bv.y);
+          imma_u8s8(ac[0][j], a0 & msk, a1 & msk, a2 & msk, a3 & msk, bv.x, bv.y);
+          if (phasB) imma_u8s8(ac[1][j], b0 & msk, b1 & msk, b2 & msk, b3 & msk, bv.x, bv.y);
         }
       }
       const float2 w = *reinterpret_cast<const float2*>(wts + (pc * NT + nt) * 8 + 2 * t);
 #pragma unroll
       for (int a = 0; a < 2; ++a) {
-        accf[a][nt][0] = fmaf((float)ac[a][0], w.x, accf[a][nt][0]);
-        accf[a][nt][1] = fmaf((float)ac[a][1], w.y, accf[a][nt][1]);
-        accf[a][nt][2] = fmaf((float)ac[a][2], w.x, accf[a][nt][2]);
-        accf[a][nt][3] = fmaf((float)ac[a][3], w.y, accf[a][nt][3]);
+        accf[a][nt][0] = fmaf((float)(ac[a][0][0] + ac[a][1][0]), w.x, accf[a][nt][0]);
+        accf[a][nt][1] = fmaf((float)(ac[a][0][1] + ac[a][1][1]), w.y, accf[a][nt][1]);
+        accf[a][nt][2] = fmaf((float)(ac[a][0][2] + ac[a][1][2]), w.x, accf[a][nt][2]);
+        accf[a][nt][3] = fmaf((float)(ac[a][0][3] + ac[a][1][3]), w.y, accf[a][nt][3]);
       }
     }
     // end of this pair's chunks: park the pair's partial in the warp's slot
@@ -481,18 +521,6 @@ static int sm_count() {
   return cached[dev];
 }
 
-static size_t g8_smem(int nt, int sc, int batch, int xs_floats) {
-  return (size_t)nt * sc * g8::kFragBytesPerChunk +
-         (size_t)g8::kWarps * g8::kMaxPairsPerWarp * g8::kSlotFloatsPerNT * nt * 4 +
-         (size_t)batch * xs_floats * 4 + (size_t)g8::kMaxTokens * 128 * 4 +
-         (size_t)sc * nt * 8 * 4 + (size_t)sc * batch * 4;
-}
-
-static int xs_floats_for(int sc, int d, int D, int Bh) {
-  const int span = (sc * 512 / D + 2) * d;
-  return Bh > 0 ? ((span + Bh - 1) / Bh + 1) * Bh : span;
-}
-
 G8Plan plan_gemv_i8(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, int32_t D,
                     int32_t Bh) {
   (void)K;
@@ -503,64 +531,97 @@ G8Plan plan_gemv_i8(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, i
   p.nt = ntok <= 1 ? 1 : ntok <= 2 ? 2 : 4;
   p.nchunk = (int)((L + 511) / 512);
   const int sms = sm_count();
-  // about 10 chunks per slice for one token; fewer when the fragments of several tokens or a
-  // large whitening block make the shared memory tight
-  int sc = std::max(1, 10 / p.nt);
-  while (sc > 1 && g8_smem(p.nt, sc, batch, xs_floats_for(sc, d, D, Bh)) > 200 * 1024) --sc;
-  p.S = (p.nchunk + sc - 1) / sc;
+  // about 10 chunks (40 KB of fragments per token pair) per slice
+  const int sc0 = std::max(1, 10 / p.nt);
+  p.S = (p.nchunk + sc0 - 1) / sc0;
   p.sc = (p.nchunk + p.S - 1) / p.S;
-  p.xs_floats = xs_floats_for(p.sc, d, D, Bh);
   p.R = std::max(1, std::min(sms / std::min(p.S, sms), (N + 31) / 32));
   p.nctas = p.S * p.R;
   // a warp's run must touch at most kMaxPairsPerWarp pairs: ceil(npair/16) + 1 <= 3
   const int npair = ((N + p.R - 1) / p.R + 31) / 32;
   if ((npair + g8::kWarps - 1) / g8::kWarps + 1 > g8::kMaxPairsPerWarp) p.ok = false;
-  p.smem = g8_smem(p.nt, p.sc, batch, p.xs_floats);
-  p.ok = p.ok && p.smem <= 220 * 1024;
+  p.smem = (size_t)p.nt * p.sc * g8::kFragBytesPerChunk +
+           (size_t)g8::kWarps * g8::kMaxPairsPerWarp * g8::kSlotFloatsPerNT * p.nt * 4 +
+           (size_t)p.sc * p.nt * 8 * 4;
+  const int span = (512 / D + 2) * d;
+  p.xs_floats = Bh > 0 ? ((span + Bh - 1) / Bh + 1) * Bh : span;
+  p.prep_smem = ((size_t)batch * p.xs_floats + (size_t)batch * 576 + 1024) * 4;
+  p.frag_bytes = (size_t)p.S * p.nt * p.sc * g8::kFragBytesPerChunk;
+  p.wtab_bytes = (size_t)p.nchunk * p.nt * 8 * 4;
+  p.csum_bytes = (size_t)p.nchunk * batch * 4;
+  p.ok = p.ok && p.smem <= 220 * 1024 && p.prep_smem <= 200 * 1024;
   return p;
 }
 
 template <int NT>
-static cudaError_t launch_nt(const G8Plan& pl, const G8Params& P, cudaStream_t st) {
-  static int smem_set[64];
-  cudaError_t e = ensure_smem((const void*)gemv_i8_kernel<NT>, pl.smem, smem_set);
+static cudaError_t launch_nt(const G8Plan& pl, const PrepParams& Q, const G8Params& P,
+                             cudaStream_t st) {
+  static int prep_set[64], smem_set[64];
+  cudaError_t e = ensure_smem((const void*)gemv_i8_prep_kernel<NT>, pl.prep_smem, prep_set);
   if (e != cudaSuccess) return e;
-  gemv_i8_kernel<NT><<<pl.nctas, g8::kThreads, pl.smem, st>>>(P);
+  e = ensure_smem((const void*)gemv_i8_kernel<NT>, pl.smem, smem_set);
+  if (e != cudaSuccess) return e;
+  gemv_i8_prep_kernel<NT><<<pl.nchunk, kPrepThreads, pl.prep_smem, st>>>(Q);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.nctas);
+  cfg.blockDim = dim3(g8::kThreads);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gemv_i8_kernel<NT>, P);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemv_i8(const G8Plan& pl, const void* x, int xdt, int32_t batch, int32_t K,
                            Whiten T, const float* M, int32_t d, int32_t D, int64_t L,
                            const uint32_t* packed, int64_t row_bytes, int32_t N, const void* s,
-                           int sdt, float* y, float* partials, uint32_t* counters,
-                           cudaStream_t st) {
+                           int sdt, float* y, void* scratch, float* partials,
+                           uint32_t* counters, cudaStream_t st) {
+  uint8_t* sp = static_cast<uint8_t*>(scratch);
+  PrepParams Q{};
+  Q.x = x;
+  Q.xdt = xdt;
+  Q.batch = batch;
+  Q.K = K;
+  Q.T = T;
+  Q.M = M;
+  Q.d = d;
+  Q.D = D;
+  Q.L = L;
+  Q.nchunk = pl.nchunk;
+  Q.sc = pl.sc;
+  Q.xs_floats = pl.xs_floats;
+  Q.frags = reinterpret_cast<uint2*>(sp);
+  Q.wtab = reinterpret_cast<float*>(sp + pl.frag_bytes);
+  Q.csum = reinterpret_cast<float*>(sp + pl.frag_bytes + pl.wtab_bytes);
   G8Params P{};
-  P.x = x;
-  P.xdt = xdt;
-  P.batch = batch;
-  P.K = K;
-  P.T = T;
-  P.M = M;
-  P.d = d;
-  P.D = D;
-  P.L = L;
   P.packed = reinterpret_cast<const uint8_t*>(packed);
   P.row_bytes = row_bytes;
   P.N = N;
   P.s = s;
   P.sdt = sdt;
   P.y = y;
+  P.batch = batch;
+  P.frags = Q.frags;
+  P.wtab = Q.wtab;
+  P.csum = Q.csum;
   P.partials = partials;
   P.counters = counters;
   P.nchunk = pl.nchunk;
   P.sc = pl.sc;
   P.S = pl.S;
   P.R = pl.R;
-  P.xs_floats = pl.xs_floats;
   switch (pl.nt) {
-    case 1: return launch_nt<1>(pl, P, st);
-    case 2: return launch_nt<2>(pl, P, st);
-    default: return launch_nt<4>(pl, P, st);
+    case 1: return launch_nt<1>(pl, Q, P, st);
+    case 2: return launch_nt<2>(pl, Q, P, st);
+    default: return launch_nt<4>(pl, Q, P, st);
   }
 }
 

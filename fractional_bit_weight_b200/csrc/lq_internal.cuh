@@ -71,25 +71,31 @@ cudaError_t launch_gemv(const GemvPlan& p, const float* z, int64_t L, int32_t ba
                         int sdt, float* y, float* partials, uint32_t* counters,
                         cudaStream_t st);
 
-// Plan of the int8 tensor-core GEMV (batch <= 8): S K-slices x R row ranges, one CTA each.
+// Plan of the int8 tensor-core GEMV (batch <= 8): a prep kernel per 512-bit chunk, then
+// S K-slices x R row ranges, one CTA each.
 struct G8Plan {
   bool ok;
-  int nt;          // 8-column MMA tiles (2 tokens each)
-  int nchunk;      // 512-bit chunks per row
-  int sc;          // chunks per slice
-  int S;           // slices
-  int R;           // row ranges
-  int nctas;       // S * R
-  int xs_floats;   // whitening scratch per token
-  size_t smem;     // dynamic shared memory per CTA
+  int nt;             // 8-column MMA tiles (2 tokens each)
+  int nchunk;         // 512-bit chunks per row
+  int sc;             // chunks per slice
+  int S;              // slices
+  int R;              // row ranges
+  int nctas;          // S * R
+  int xs_floats;      // whitening scratch per token (prep)
+  size_t smem;        // gemv dynamic shared memory per CTA
+  size_t prep_smem;   // prep dynamic shared memory per CTA
+  size_t frag_bytes;  // scratch: B fragments
+  size_t wtab_bytes;  // scratch: per-chunk column weights
+  size_t csum_bytes;  // scratch: per-chunk sums of z
 };
 G8Plan plan_gemv_i8(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, int32_t D,
                     int32_t Bh);
-// partials: [S][batch][N] floats and counters: [R] zeroed uint32 (both unused when S == 1)
+// scratch: frag_bytes + wtab_bytes + csum_bytes bytes (16-byte aligned); partials:
+// [S][batch][N] floats and counters: [R] zeroed uint32 (both unused when S == 1)
 cudaError_t launch_gemv_i8(const G8Plan& pl, const void* x, int xdt, int32_t batch, int32_t K,
                            Whiten T, const float* M, int32_t d, int32_t D, int64_t L,
                            const uint32_t* packed, int64_t row_bytes, int32_t N, const void* s,
-                           int sdt, float* y, float* partials, uint32_t* counters,
-                           cudaStream_t st);
+                           int sdt, float* y, void* scratch, float* partials,
+                           uint32_t* counters, cudaStream_t st);
 
 }  // namespace lq

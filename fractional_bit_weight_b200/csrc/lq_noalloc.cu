@@ -17,7 +17,8 @@
 namespace {
 
 // The scratch of every lq_gemm_noalloc call on a device: split-K completion counters at offset
-// 0 (they must start at zero; the kernel returns them to zero), then the fp32 slice partials.
+// 0 (they must start at zero; the kernel returns them to zero), then the activation fragments
+// that each call's first kernel writes, then the fp32 slice partials.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[LQ_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
@@ -89,23 +90,26 @@ extern "C" lq_status lq_gemm_noalloc(const void* x, lq_dtype xdt, int32_t batch,
   const int64_t L = ((int64_t)K + d - 1) / d * D;
   const int64_t row_bytes = ((L + 7) / 8 + 15) / 16 * 16;
   const lq::G8Plan pl = lq::plan_gemv_i8(batch, L, N, K, d, D, w.block);
-  if (!pl.ok) return reject(LQ_EUNSUPPORTED, "lq_gemm_noalloc: shape not supported by the GEMV path");
+  const size_t prep_bytes = (pl.frag_bytes + pl.wtab_bytes + pl.csum_bytes + 255) / 256 * 256;
   const size_t partial_bytes = pl.S > 1 ? (size_t)pl.S * batch * N * sizeof(float) : 0;
-  const size_t need = kCounterBytes + partial_bytes;
+  const size_t need = kCounterBytes + prep_bytes + partial_bytes;
   if ((size_t)pl.R * sizeof(uint32_t) > kCounterBytes || need > LQ_NOALLOC_SCRATCH_BYTES)
     return reject(LQ_EINVAL,
                   "lq_gemm_noalloc: this shape needs %zu bytes of scratch, more than the "
                   "LQ_NOALLOC_SCRATCH_BYTES = %zu the library holds; use lq_gemm with a workspace",
                   need, (size_t)LQ_NOALLOC_SCRATCH_BYTES);
+  if (!pl.ok) return reject(LQ_EUNSUPPORTED, "lq_gemm_noalloc: shape not supported by the GEMV path");
 
   void* scratch = nullptr;
   st = scratch_for_current_device(&scratch);
   if (st != LQ_OK) return st;
   uint8_t* base = static_cast<uint8_t*>(scratch);
   uint32_t* counters = reinterpret_cast<uint32_t*>(base);
-  float* partials = reinterpret_cast<float*>(base + kCounterBytes);
+  void* prep = base + kCounterBytes;
+  float* partials = reinterpret_cast<float*>(base + kCounterBytes + prep_bytes);
   cudaError_t e = lq::launch_gemv_i8(pl, x, (int)xdt, batch, K, w, M, d, D, L, packed, row_bytes,
-                                     N, s, (int)sdt, y, partials, counters, (cudaStream_t)stream);
+                                     N, s, (int)sdt, y, prep, partials, counters,
+                                     (cudaStream_t)stream);
   if (e != cudaSuccess)
     return reject(LQ_ECUDA, "lq_gemm_noalloc: %s", cudaGetErrorString(e));
   return LQ_OK;
