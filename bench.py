@@ -232,9 +232,9 @@ def _x_tensor(layer):
 
 
 def kernels_per_step(batch):
-    """Kernels one lq_gemm call launches: the fused int8 GEMV (batch <= 8), else the lift
-    prologue plus the fp32 GEMV."""
-    return 1 if batch <= 8 else 2
+    """Kernels one lq_gemm call launches: a prologue (whitening + lift) and the contraction,
+    on every path (int8 GEMV for batch <= 8, tcgen05 GEMM for batch >= 64, fp32 GEMV between)."""
+    return 2
 
 
 def time_steps(fn, steps, warmup, ws, graph_block=None):
@@ -347,10 +347,12 @@ def main():
     else:
         metric, value, unit = "lq_prefill_gemm_TFLOPs", tflops, "TFLOP/s"
         achieved = wl.flops() / per_step / 1e12
-        peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+        # the burst figure: the timed region is short and the clocks stay at their maximum
+        # (the sampled clocks are in the same line); fp16 dense rate = bf16 dense rate
+        peak = float(peaks.get("bf16_tflops", peaks.get("bf16_tflops_sustained")))
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
-                "peak_source": f"{peak_src} bf16_tflops_sustained (fp16 dense = bf16 dense)"}
+                "peak_source": f"{peak_src} bf16_tflops (burst; fp16 dense = bf16 dense)"}
 
     out = {
         "metric": metric, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,

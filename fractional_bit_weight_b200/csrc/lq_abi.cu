@@ -70,22 +70,27 @@ lq_status make_whiten(const lq_whiten_desc* T, int32_t K, lq::Whiten* out) {
 
 // Workspace layout of lq_gemm (byte offsets, all 256-aligned).
 struct WsLayout {
-  int path;          // 0: int8 tensor-core GEMV (batch <= 8); 1: fp32 GEMV over z
+  int path;          // 0: int8 tensor-core GEMV (batch <= 8); 1: fp32 GEMV over z;
+                     // 2: tcgen05 GEMM (batch >= lq::kTcMinBatch)
   size_t counters;   // uint32 completion counters of the split-K reduction
   size_t z;          // path 0: prep output (fragments, weights, sums); path 1: float z [batch][L]
   size_t partials;   // float [slices][batch][N]
   size_t total;
   lq::GemvPlan gemv;
   lq::G8Plan g8;
+  lq::TcPlan tc;
 };
 
 WsLayout layout_gemm(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D, int32_t Bh) {
   WsLayout w{};
   const int64_t L = lifted_bits(K, d, D);
   w.g8 = lq::plan_gemv_i8(batch, L, N, K, d, D, Bh);
-  w.path = w.g8.ok ? 0 : 1;
+  w.tc = lq::plan_gemm_tc(batch, L, N, K, d);
+  w.path = w.g8.ok ? 0 : (w.tc.ok ? 2 : 1);
   size_t ncounters = 0, npartials = 0, nz = 0;
-  if (w.path == 0) {
+  if (w.path == 2) {
+    nz = (w.tc.z_bytes + w.tc.scale_bytes + 3) / 4;   // fp16 z, then the token scales
+  } else if (w.path == 0) {
     ncounters = (size_t)w.g8.R;
     npartials = w.g8.S > 1 ? (size_t)w.g8.S * batch * N : 0;
     nz = (w.g8.frag_bytes + w.g8.wtab_bytes + w.g8.csum_bytes + 3) / 4;   // prep output
@@ -251,6 +256,12 @@ lq_status lq_gemm(const void* x, lq_dtype xdt, int32_t batch, const lq_whiten_de
   const int64_t L = lifted_bits(K, d, D);
   uint32_t* counters = reinterpret_cast<uint32_t*>(ws + lay.counters);
   float* partials = reinterpret_cast<float*>(ws + lay.partials);
+  if (lay.path == 2) {
+    cudaError_t e = lq::launch_gemm_tc(lay.tc, x, (int)xdt, batch, K, w, M, d, D, L, packed,
+                                       row_stride_bytes(K, d, D), N, s, (int)sdt, y, ws + lay.z,
+                                       reinterpret_cast<uint32_t*>(ws), cs);
+    return e == cudaSuccess ? LQ_OK : cuda_fail(e, "lq_gemm (tensor-core gemm)");
+  }
   if (lay.path == 0) {
     cudaError_t e = lq::launch_gemv_i8(lay.g8, x, (int)xdt, batch, K, w, M, d, D, L, packed,
                                        row_stride_bytes(K, d, D), N, s, (int)sdt, y, ws + lay.z,

@@ -98,4 +98,25 @@ cudaError_t launch_gemv_i8(const G8Plan& pl, const void* x, int xdt, int32_t bat
                            int sdt, float* y, void* scratch, float* partials,
                            uint32_t* counters, cudaStream_t st);
 
+// Plan of the tensor-core GEMM (batch >= kTcMinBatch): a whiten + lift prologue writing fp16
+// z with a per-token power-of-two scale, then a persistent tcgen05 kernel over 128-token x
+// 256-row tiles.
+constexpr int32_t kTcMinBatch = 64;
+struct TcPlan {
+  bool ok;
+  int Lp;              // lifted length padded to the 64-coordinate stage
+  int nks;             // stages per tile (Lp / 64)
+  int tiles_n, tiles_m, tiles;
+  size_t smem;         // GEMM dynamic shared memory per CTA
+  size_t pro_smem;     // prologue dynamic shared memory per CTA
+  size_t z_bytes;      // scratch: fp16 z [batch][Lp]
+  size_t scale_bytes;  // scratch: float 2^-e [batch], right after z
+};
+TcPlan plan_gemm_tc(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d);
+// scratch: z_bytes + scale_bytes bytes, 256-byte aligned; status: the workspace status word
+cudaError_t launch_gemm_tc(const TcPlan& pl, const void* x, int xdt, int32_t batch, int32_t K,
+                           Whiten T, const float* M, int32_t d, int32_t D, int64_t L,
+                           const uint32_t* packed, int64_t row_bytes, int32_t N, const void* s,
+                           int sdt, float* y, void* scratch, uint32_t* status, cudaStream_t st);
+
 }  // namespace lq

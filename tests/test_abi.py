@@ -60,6 +60,18 @@ def test_workspace_bytes(L):
     assert lq.gemm_workspace_bytes(1, 4096, 4096, 10, 33) == 0
 
 
+def _r256(n):
+    return -(-n // 256) * 256
+
+
+@pytest.mark.parametrize("batch,K,N,d,D", [(64, 8192, 28672, 10, 24), (2048, 8192, 28672, 10, 24),
+                                           (200, 512, 600, 10, 24), (300, 96, 513, 16, 32)])
+def test_workspace_of_tensor_core_path(L, batch, K, N, d, D):
+    """batch >= 64: a 256-byte header, fp16 z [batch][L padded to 64], then batch fp32 scales."""
+    Lp = -(-lq.lifted_bits(K, d, D) // 64) * 64
+    assert lq.gemm_workspace_bytes(batch, K, N, d, D) == 256 + _r256(batch * Lp * 2 + batch * 4)
+
+
 def _ptr(v):
     return ctypes.c_void_p(v)
 
