@@ -37,7 +37,10 @@ FALLBACK_BF16_TFLOPS = 1590.0
 WORKLOADS = {
     "llama2_7b_qproj_b1": (2, 0, "gemv"),
     "llama3_70b_gateup_b1": (3, 0, "gemv"),
+    "llama3_70b_gateup_b4": (3, 1, "gemv"),
     "llama3_70b_gateup_b16": (3, 2, "gemv"),
+    "llama3_70b_down_b4": (3, 4, "gemv"),
+    "llama3_70b_down_b16": (3, 5, "gemv"),
     "llama3_70b_down_b1": (3, 3, "gemv"),
     "sweep_d10D24_b1": (4, 8, "gemv"),
     "prefill_b2048": (5, 0, "gemm"),
@@ -231,10 +234,9 @@ def _x_tensor(layer):
     return torch.from_numpy(np.ascontiguousarray(layer.x_raw))
 
 
-def kernels_per_step(batch):
-    """Kernels one lq_gemm call launches: a prologue (whitening + lift) and the contraction,
-    on every path (int8 GEMV for batch <= 8, tcgen05 GEMM for batch >= 64, fp32 GEMV between)."""
-    return 2
+def kernels_per_step(wl):
+    """Kernels one lq_gemm call launches for this workload, as the library reports it."""
+    return lq.gemm_launches(wl.batch, wl.K, wl.N, wl.d, wl.D, wl.block)
 
 
 def time_steps(fn, steps, warmup, ws, graph_block=None):
@@ -365,7 +367,7 @@ def main():
                    "l2": f"rotating {wl.ncopies} copies of the packed weights "
                          f"({wl.ncopies * wl.stored_bytes / 1e6:.0f} MB > L2)"},
         "roofline": roof,
-        "gpu_launches": kernels_per_step(wl.batch) * args.steps,
+        "gpu_launches": kernels_per_step(wl) * args.steps,
         "timing": "CUDA graphs of the steps, replayed; CUDA events on the launching stream",
         "clocks": clk.summary(),
     }

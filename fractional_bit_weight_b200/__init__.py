@@ -13,7 +13,8 @@ import torch
 
 __all__ = [
     "LQError", "lib", "abi_version", "lifted_bits", "row_stride_bytes", "pack", "unpack",
-    "whiten", "lift", "gemm_workspace_bytes", "gemm", "gemm_noalloc", "new_workspace",
+    "whiten", "lift", "gemm_workspace_bytes", "gemm_launches", "gemm", "gemm_noalloc",
+    "new_workspace",
     "device_status", "NOALLOC_SCRATCH_BYTES",
 ]
 
@@ -27,7 +28,8 @@ LQ_F32, LQ_F16, LQ_BF16 = 0, 1, 2
 _DTYPES = {torch.float32: LQ_F32, torch.float16: LQ_F16, torch.bfloat16: LQ_BF16}
 
 EXPORTS = ("lq_abi_version", "lq_lifted_bits", "lq_row_stride_bytes", "lq_pack", "lq_unpack",
-           "lq_whiten", "lq_lift", "lq_gemm_workspace_bytes", "lq_gemm", "lq_gemm_noalloc",
+           "lq_whiten", "lq_lift", "lq_gemm_workspace_bytes", "lq_gemm_launches", "lq_gemm",
+           "lq_gemm_noalloc",
            "lq_device_status", "lq_status_string", "lq_last_error")
 
 
@@ -57,6 +59,7 @@ def _declare(L):
         "lq_whiten": ([vp, ctypes.c_int, i32, i32, dp, vp, vp], ctypes.c_int),
         "lq_lift": ([vp, ctypes.c_int, i32, i32, dp, vp, i32, i32, vp, vp], ctypes.c_int),
         "lq_gemm_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
+        "lq_gemm_launches": ([i32, i32, i32, i32, i32, i32], i32),
         "lq_gemm": ([vp, ctypes.c_int, i32, dp, vp, vp, vp, ctypes.c_int, i32, i32, i32, i32, vp,
                      vp, sz, vp], ctypes.c_int),
         "lq_gemm_noalloc": ([vp, ctypes.c_int, i32, dp, vp, vp, vp, ctypes.c_int, i32, i32, i32,
@@ -176,6 +179,11 @@ def lift(x, M, d, D, sign=None, chan_scale=None, block=0, out=None, stream=None)
 
 def gemm_workspace_bytes(batch, K, N, d, D):
     return int(lib().lq_gemm_workspace_bytes(batch, K, N, d, D))
+
+
+def gemm_launches(batch, K, N, d, D, block=0):
+    """Kernels one lq_gemm call launches for this shape (host-only query)."""
+    return int(lib().lq_gemm_launches(batch, K, N, d, D, block))
 
 
 def new_workspace(batch, K, N, d, D, device="cuda"):

@@ -71,13 +71,16 @@ lq_status make_whiten(const lq_whiten_desc* T, int32_t K, lq::Whiten* out) {
 // Workspace layout of lq_gemm (byte offsets, all 256-aligned).
 struct WsLayout {
   int path;          // 0: int8 tensor-core GEMV (batch <= 8); 1: fp32 GEMV over z;
-                     // 2: tcgen05 GEMM (batch >= lq::kTcMinBatch)
+                     // 2: tcgen05 GEMM (batch >= lq::kTcMinBatch); 3: the int8 GEMV once per
+                     // group of gs tokens (when no single-launch plan fits)
   size_t counters;   // uint32 completion counters of the split-K reduction
   size_t z;          // path 0: prep output (fragments, weights, sums); path 1: float z [batch][L]
   size_t partials;   // float [slices][batch][N]
   size_t total;
   lq::GemvPlan gemv;
   lq::G8Plan g8;
+  lq::G8Plan g8r;    // path 3: the plan of the last, smaller group
+  int gs;            // path 3: tokens per group
   lq::TcPlan tc;
 };
 
@@ -86,9 +89,39 @@ WsLayout layout_gemm(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D, 
   const int64_t L = lifted_bits(K, d, D);
   w.g8 = lq::plan_gemv_i8(batch, L, N, K, d, D, Bh);
   w.tc = lq::plan_gemm_tc(batch, L, N, K, d);
-  w.path = w.g8.ok ? 0 : (w.tc.ok ? 2 : 1);
+  w.path = w.g8.ok ? 0 : (w.tc.ok && batch >= lq::kTcMinBatch ? 2 : 1);
+  // no single-launch GEMV fits: the largest token group whose int8 GEMV plan does, once per
+  // group
+  for (int32_t gs : {8, 4, 2, 1}) {
+    if (w.path != 1 || gs >= batch) continue;
+    w.g8 = lq::plan_gemv_i8(gs, L, N, K, d, D, Bh);
+    w.g8r = batch % gs ? lq::plan_gemv_i8(batch % gs, L, N, K, d, D, Bh) : w.g8;
+    if (w.g8.ok && w.g8r.ok) {
+      w.path = 3;
+      w.gs = gs;
+    }
+  }
+  // below kTcMinBatch tokens the tensor-core GEMM still wins once the groups are many: rough
+  // B200 costs, each group streaming the codes at ~2 TB/s plus ~6 us, each wave of 128 x 256
+  // tiles ~0.7 us per 64-coordinate stage
+  if (w.path == 3 && w.tc.ok) {
+    const double groups = (double)((batch + w.gs - 1) / w.gs);
+    const double gemv_s = groups * ((double)N * (double)row_stride_bytes(K, d, D) / 2.0e12 + 6e-6);
+    const int sms = 148;
+    const double tc_s = (double)((w.tc.tiles + sms - 1) / sms) * w.tc.nks * 0.7e-6 + 10e-6;
+    if (tc_s < gemv_s) w.path = 2;
+  }
+  if (w.path == 1 && w.tc.ok && batch > 8) w.path = 2;
   size_t ncounters = 0, npartials = 0, nz = 0;
-  if (w.path == 2) {
+  if (w.path == 3) {
+    // the groups run one after the other on the stream and share the scratch
+    for (const lq::G8Plan* g : {&w.g8, &w.g8r}) {
+      const int nb = g == &w.g8 ? w.gs : (batch % w.gs ? batch % w.gs : w.gs);
+      ncounters = std::max(ncounters, (size_t)g->R);
+      npartials = std::max(npartials, g->S > 1 ? (size_t)g->S * nb * N : (size_t)0);
+      nz = std::max(nz, (g->frag_bytes + g->wtab_bytes + g->csum_bytes + 3) / 4);
+    }
+  } else if (w.path == 2) {
     nz = (w.tc.z_bytes + w.tc.scale_bytes + 3) / 4;   // fp16 z, then the token scales
   } else if (w.path == 0) {
     ncounters = (size_t)w.g8.R;
@@ -228,6 +261,15 @@ size_t lq_gemm_workspace_bytes(int32_t batch, int32_t K, int32_t N, int32_t d, i
   return best;
 }
 
+int32_t lq_gemm_launches(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D,
+                         int32_t block) {
+  if (!valid_code(K, d, D) || batch < 1 || batch > kMaxBatch || N < 1 || K > kMaxK) return 0;
+  if (block < 0 || block > LQ_MAX_HADAMARD || (block & (block - 1)) != 0) return 0;
+  const WsLayout lay = layout_gemm(batch, K, N, d, D, block);
+  // every path: a prologue kernel and a contraction kernel, per token group on path 3
+  return lay.path == 3 ? 2 * ((batch + lay.gs - 1) / lay.gs) : 2;
+}
+
 lq_status lq_gemm(const void* x, lq_dtype xdt, int32_t batch, const lq_whiten_desc* T,
                   const uint32_t* packed, const float* M, const void* s, lq_dtype sdt,
                   int32_t d, int32_t D, int32_t K, int32_t N, float* y, void* workspace,
@@ -267,6 +309,17 @@ lq_status lq_gemm(const void* x, lq_dtype xdt, int32_t batch, const lq_whiten_de
                                        row_stride_bytes(K, d, D), N, s, (int)sdt, y, ws + lay.z,
                                        partials, counters, cs);
     return e == cudaSuccess ? LQ_OK : cuda_fail(e, "lq_gemm (int8 gemv)");
+  }
+  if (lay.path == 3) {
+    for (int32_t t0 = 0; t0 < batch; t0 += lay.gs) {
+      const int32_t nb = std::min<int32_t>(lay.gs, batch - t0);
+      const char* xt = static_cast<const char*>(x) + (size_t)t0 * K * dtype_size(xdt);
+      cudaError_t e = lq::launch_gemv_i8(nb == lay.gs ? lay.g8 : lay.g8r, xt, (int)xdt, nb, K, w, M, d,
+                                         D, L, packed, row_stride_bytes(K, d, D), N, s, (int)sdt,
+                                         y + (size_t)t0 * N, ws + lay.z, partials, counters, cs);
+      if (e != cudaSuccess) return cuda_fail(e, "lq_gemm (int8 gemv, token group)");
+    }
+    return LQ_OK;
   }
   if (lay.gemv.ntiles > 65535 || lay.gemv.ntg > 65535)
     return fail(LQ_EUNSUPPORTED, "N or batch too large for one launch");

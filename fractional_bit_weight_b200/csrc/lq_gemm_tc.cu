@@ -435,7 +435,7 @@ int sm_count() {
 
 TcPlan plan_gemm_tc(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d) {
   TcPlan p{};
-  if (batch < kTcMinBatch) return p;
+  if (batch < 1) return p;
   const int64_t Kp = ((int64_t)K + d - 1) / d * d;
   p.pro_smem = (size_t)(LQ_MAX_D * LQ_MAX_D + Kp) * sizeof(float);
   if (p.pro_smem > 200 * 1024) return p;

@@ -98,7 +98,8 @@ cudaError_t launch_gemv_i8(const G8Plan& pl, const void* x, int xdt, int32_t bat
                            int sdt, float* y, void* scratch, float* partials,
                            uint32_t* counters, cudaStream_t st);
 
-// Plan of the tensor-core GEMM (batch >= kTcMinBatch): a whiten + lift prologue writing fp16
+// Plan of the tensor-core GEMM (always used from kTcMinBatch tokens, below that when it is
+// expected to beat the int8 GEMV run per token group): a whiten + lift prologue writing fp16
 // z with a per-token power-of-two scale, then a persistent tcgen05 kernel over 128-token x
 // 256-row tiles.
 constexpr int32_t kTcMinBatch = 64;

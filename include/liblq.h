@@ -116,6 +116,12 @@ LQ_API lq_status lq_lift(const void* x, lq_dtype xdt, int32_t batch, int32_t K,
 /* Workspace bytes lq_gemm needs for this shape (0 on invalid sizes). */
 LQ_API size_t lq_gemm_workspace_bytes(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D);
 
+/* Number of kernels one lq_gemm call launches for this shape and Hadamard block (0 on invalid
+ * sizes). Host-only, touches no device. No counterpart on the pages: it lets a caller account
+ * for launches (graph sizing, profiling). */
+LQ_API int32_t lq_gemm_launches(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D,
+                                int32_t block);
+
 /* The decode operator, y = s . (W T(x)) (paper sec. 3 intro: o = diag(s) W (M T a);
  * review: diag(s) W_q (T* a)).
  *   x       [batch][K] of dtype xdt (f32, f16 or bf16)

@@ -64,6 +64,15 @@ def _r256(n):
     return -(-n // 256) * 256
 
 
+def test_gemm_launches(L):
+    assert lq.gemm_launches(1, 4096, 4096, 10, 24, 256) == 2        # int8 GEMV
+    assert lq.gemm_launches(2048, 8192, 28672, 10, 24, 256) == 2    # tcgen05 GEMM
+    n16 = lq.gemm_launches(16, 28672, 8192, 10, 24, 256)            # token groups
+    assert n16 >= 4 and n16 % 2 == 0
+    assert lq.gemm_launches(0, 4096, 4096, 10, 24, 256) == 0
+    assert lq.gemm_launches(1, 4096, 4096, 10, 24, 3) == 0
+
+
 @pytest.mark.parametrize("batch,K,N,d,D", [(64, 8192, 28672, 10, 24), (2048, 8192, 28672, 10, 24),
                                            (200, 512, 600, 10, 24), (300, 96, 513, 16, 32)])
 def test_workspace_of_tensor_core_path(L, batch, K, N, d, D):
