@@ -325,36 +325,45 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return v;
 }
 
+constexpr int kLiftChunk = 4096;   // lifted coordinates per pass of the prologue
+
 // One CTA per token: zh[t][0 .. Lp) fp16 (word-interleaved order, zero beyond L) and
-// inv_scale[t] = 2^-e.
+// inv_scale[t] = 2^-e. Dynamic shared memory: M in rows of D4 = D rounded up to 4 columns
+// (zero beyond D), xt zero-padded to Kp, then one pass of natural-order z.
 __global__ void __launch_bounds__(512)
     lift_f16_kernel(const void* __restrict__ x, int xdt, int K, Whiten T,
                     const float* __restrict__ M, int d, int D, int Kp, int64_t L, int Lp,
                     __half* __restrict__ zh, float* __restrict__ inv_scale) {
-  extern __shared__ float sm[];
+  extern __shared__ __align__(16) float sm[];
   __shared__ float red[32];
-  float* sM = sm;                      // [d][D]
-  float* sx = sm + LQ_MAX_D * LQ_MAX_D;  // xt, zero-padded to Kp
+  float* sM = sm;                          // [d][D4]
+  float* sx = sm + LQ_MAX_D * LQ_MAX_D;    // xt, zero-padded to Kp
+  float* zc = sx + ((Kp + 3) & ~3);        // z of one pass, natural order
   const int t = blockIdx.x;
+  const int tid = threadIdx.x;
   const int64_t row = (int64_t)t * K;
-  for (int i = threadIdx.x; i < d * D; i += blockDim.x) sM[i] = M[i];
+  const int D4 = (D + 3) & ~3;
+  for (int k = tid; k < d * D4; k += blockDim.x) {
+    const int i = k / D4, j = k - i * D4;
+    sM[k] = j < D ? M[i * D + j] : 0.f;
+  }
   if (T.block > 0) {
     whiten_blocks_smem(x, xdt, row, K, T, 0, K / T.block, sx);   // ends with a barrier
   } else {
-    for (int k = threadIdx.x; k < K; k += blockDim.x) sx[k] = load_as_f32(x, xdt, row + k);
+    for (int k = tid; k < K; k += blockDim.x) sx[k] = load_as_f32(x, xdt, row + k);
   }
-  for (int k = K + threadIdx.x; k < Kp; k += blockDim.x) sx[k] = 0.f;
+  for (int k = K + tid; k < Kp; k += blockDim.x) sx[k] = 0.f;
   __syncthreads();
 
   // |z[g*D+j]| <= max|xt| * max_j sum_i |M[i][j]|: a power-of-two scale that maps this bound
   // to at most 2^14 keeps every fp16 value finite and normal-range for any input.
   float amax = 0.f;
-  for (int k = threadIdx.x; k < K; k += blockDim.x) amax = fmaxf(amax, fabsf(sx[k]));
+  for (int k = tid; k < K; k += blockDim.x) amax = fmaxf(amax, fabsf(sx[k]));
   amax = block_max(amax, red);
   float cs = 0.f;
-  for (int j = threadIdx.x; j < D; j += blockDim.x) {
+  for (int j = tid; j < D; j += blockDim.x) {
     float c = 0.f;
-    for (int i = 0; i < d; ++i) c += fabsf(sM[i * D + j]);
+    for (int i = 0; i < d; ++i) c += fabsf(sM[i * D4 + j]);
     cs = fmaxf(cs, c);
   }
   const float cmax = block_max(cs, red);
@@ -366,35 +375,61 @@ __global__ void __launch_bounds__(512)
     sh = min(120, max(-120, 14 - ex));
   }
   const float scale = ldexpf(1.f, sh);
-  if (threadIdx.x == 0) inv_scale[t] = ldexpf(1.f, -sh);
+  if (tid == 0) inv_scale[t] = ldexpf(1.f, -sh);
 
-  // 8 consecutive stored positions per item: positions q0 + 2i + h hold coordinate q0 + i + 16h
   __half* zrow = zh + (int64_t)t * Lp;
-  const int items = Lp / 8;
-  for (int it = threadIdx.x; it < items; it += blockDim.x) {
-    const int pos0 = it * 8;
-    const int64_t q0 = pos0 & ~31;
-    const int i0 = (pos0 & 31) >> 1;
-    uint32_t packed[4];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      float v2[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int64_t q = q0 + i0 + r + 16 * h;
-        float acc = 0.f;
-        if (q < L) {
-          const int g = (int)(q / D);
-          const int j = (int)(q - (int64_t)g * D);
-          const float* xg = sx + (int64_t)g * d;
-          for (int i = 0; i < d; ++i) acc = fmaf(sM[i * D + j], xg[i], acc);
+  const int nb = D4 >> 2;
+  for (int cq = 0; cq < Lp; cq += kLiftChunk) {
+    const int qe = min(cq + kLiftChunk, Lp);             // stored positions [cq, qe)
+    const int qv = (int)min((int64_t)qe, L);             // coordinates with a value
+    // natural-order z of [cq, qv): a thread takes 4 columns of one group (lanes: consecutive
+    // groups, same columns, so the 16-byte M loads are shared by the warp)
+    if (cq < qv) {
+      const int g_lo = cq / D, g_hi = (qv - 1) / D;
+      const int ng = g_hi - g_lo + 1;
+      for (int task = tid; task < ng * nb; task += blockDim.x) {
+        const int jb = task / ng, gl = task - jb * ng;
+        const int g = g_lo + gl;
+        const float* xg = sx + g * d;
+        const float* mc = sM + 4 * jb;
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 2
+        for (int i = 0; i < d; ++i) {
+          const float xv = xg[i];
+          const float4 m4 = *reinterpret_cast<const float4*>(mc + i * D4);
+          a0 = fmaf(m4.x, xv, a0);
+          a1 = fmaf(m4.y, xv, a1);
+          a2 = fmaf(m4.z, xv, a2);
+          a3 = fmaf(m4.w, xv, a3);
         }
-        v2[h] = acc * scale;
+        const int qb = g * D + 4 * jb;
+        const float av[4] = {a0, a1, a2, a3};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int q = qb + u;
+          if (4 * jb + u < D && q >= cq && q < qv) zc[q - cq] = av[u];
+        }
       }
-      const __half2 hv = __floats2half2_rn(v2[0], v2[1]);
-      packed[r] = *reinterpret_cast<const uint32_t*>(&hv);
     }
-    *reinterpret_cast<uint4*>(zrow + pos0) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    for (int ql = max(0, qv - cq) + tid; ql < qe - cq; ql += blockDim.x) zc[ql] = 0.f;
+    __syncthreads();
+    // 8 consecutive stored positions per item: positions q0 + 2i + h hold coordinate
+    // q0 + i + 16h (passes start on multiples of 32, so a word never straddles two)
+    for (int it = tid; it < (qe - cq) / 8; it += blockDim.x) {
+      const int pos0 = cq + it * 8;
+      const int q0 = pos0 & ~31;
+      const int i0 = (pos0 & 31) >> 1;
+      uint32_t packed[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float v0 = zc[q0 + i0 + r - cq] * scale;
+        const float v1 = zc[q0 + i0 + r + 16 - cq] * scale;
+        const __half2 hv = __floats2half2_rn(v0, v1);
+        packed[r] = *reinterpret_cast<const uint32_t*>(&hv);
+      }
+      *reinterpret_cast<uint4*>(zrow + pos0) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    }
+    __syncthreads();
   }
 }
 
@@ -437,7 +472,7 @@ TcPlan plan_gemm_tc(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d) {
   TcPlan p{};
   if (batch < 1) return p;
   const int64_t Kp = ((int64_t)K + d - 1) / d * d;
-  p.pro_smem = (size_t)(LQ_MAX_D * LQ_MAX_D + Kp) * sizeof(float);
+  p.pro_smem = (size_t)(LQ_MAX_D * LQ_MAX_D + ((Kp + 3) & ~3) + tc::kLiftChunk) * sizeof(float);
   if (p.pro_smem > 200 * 1024) return p;
   const int64_t Lp = (L + tc::BK - 1) / tc::BK * tc::BK;
   if (Lp > (1 << 30)) return p;
