@@ -94,18 +94,15 @@ def measured_peaks():
                 "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def csrc_digest():
-    h = hashlib.sha256()
-    d = os.path.join(ROOT, "fractional_bit_weight_b200", "csrc")
-    for name in sorted(os.listdir(d)):
-        with open(os.path.join(d, name), "rb") as f:
-            h.update(name.encode() + f.read())
-    return h.hexdigest()[:16]
+def source_digest(name):
+    """Digest of one kernel source file under fractional_bit_weight_b200/csrc."""
+    with open(os.path.join(ROOT, "fractional_bit_weight_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
 def recorded_traffic(workload):
-    """DRAM bytes per launch of the dominant kernel from a committed ncu summary, if it was
-    taken on the current kernel sources (else None)."""
+    """DRAM bytes per launch of the workload's dominant kernel from profiles/traffic.json (an
+    ncu capture), if the file defining that kernel is unchanged since (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -113,70 +110,12 @@ def recorded_traffic(workload):
     except (OSError, ValueError):
         return None
     ent = rec.get(workload)
-    if not ent or ent.get("csrc_digest") != csrc_digest():
+    try:
+        if not ent or ent.get("source_digest") != source_digest(ent["source"]):
+            return None
+    except (OSError, KeyError):
         return None
     return ent.get("dram_bytes_per_launch")
-
-
-class ClockSampler:
-    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
-
-    def __init__(self, index):
-        self.samples, self.reasons = [], set()
-        self.max_mhz = None
-        self._stop = threading.Event()
-        try:
-            import pynvml
-            pynvml.nvmlInit()
-            self._nv = pynvml
-            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
-        except Exception:
-            self._nv = None
-        self._t = threading.Thread(target=self._run, daemon=True)
-
-    def _sample(self):
-        nv = self._nv
-        self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-        r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-        names = {
-            "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap,
-            "hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
-            "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
-            "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
-            "hw_power_brake_slowdown": nv.nvmlClocksEventReasonHwPowerBrakeSlowdown,
-        }
-        for k, bit in names.items():
-            if r & bit:
-                self.reasons.add(k)
-
-    def _run(self):
-        while not self._stop.is_set():
-            try:
-                self._sample()
-            except Exception:
-                return
-            time.sleep(0.002)
-
-    def __enter__(self):
-        if self._nv is not None:
-            self._t.start()
-        return self
-
-    def __exit__(self, *a):
-        self._stop.set()
-        if self._nv is not None:
-            self._t.join()
-            try:
-                self._sample()
-            except Exception:
-                pass
-
-    def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
-        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
 # ---------------------------------------------------------------- workload on the device
