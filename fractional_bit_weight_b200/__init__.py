@@ -15,7 +15,7 @@ __all__ = [
     "LQError", "lib", "abi_version", "lifted_bits", "row_stride_bytes", "pack", "unpack",
     "whiten", "lift", "gemm_workspace_bytes", "gemm_launches", "gemm", "gemm_noalloc",
     "new_workspace",
-    "device_status", "NOALLOC_SCRATCH_BYTES",
+    "device_status", "check_wait_timeout", "NOALLOC_SCRATCH_BYTES",
 ]
 
 NOALLOC_SCRATCH_BYTES = 8 << 20   # LQ_NOALLOC_SCRATCH_BYTES
@@ -29,7 +29,7 @@ _DTYPES = {torch.float32: LQ_F32, torch.float16: LQ_F16, torch.bfloat16: LQ_BF16
 
 EXPORTS = ("lq_abi_version", "lq_lifted_bits", "lq_row_stride_bytes", "lq_pack", "lq_unpack",
            "lq_whiten", "lq_lift", "lq_gemm_workspace_bytes", "lq_gemm_launches", "lq_gemm",
-           "lq_gemm_noalloc",
+           "lq_gemm_noalloc", "lq_check_wait_timeout",
            "lq_device_status", "lq_status_string", "lq_last_error")
 
 
@@ -65,6 +65,7 @@ def _declare(L):
         "lq_gemm_noalloc": ([vp, ctypes.c_int, i32, dp, vp, vp, vp, ctypes.c_int, i32, i32, i32,
                              i32, vp, vp], ctypes.c_int),
         "lq_device_status": ([vp, ctypes.POINTER(i32), vp], ctypes.c_int),
+        "lq_check_wait_timeout": ([vp, i32, vp], ctypes.c_int),
         "lq_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "lq_last_error": ([], ctypes.c_char_p),
     }
@@ -232,6 +233,13 @@ def gemm_noalloc(x, packed, M, s, d, D, sign=None, chan_scale=None, block=0, y=N
                                  _DTYPES[s.dtype], d, D, K, N, _dev(y, "y", (torch.float32,)),
                                  _stream(stream)), "lq_gemm_noalloc")
     return y
+
+
+def check_wait_timeout(workspace, limit_ms=20, stream=None):
+    """Runs the device-side timeout check (see lq_check_wait_timeout); read the result with
+    device_status(workspace)."""
+    _check(lib().lq_check_wait_timeout(_dev(workspace, "workspace"), int(limit_ms),
+                                       _stream(stream)), "lq_check_wait_timeout")
 
 
 def device_status(workspace, stream=None):

@@ -120,6 +120,8 @@ constexpr int kPrepThreads = 512;
 // One CTA per chunk; see the file comment.
 template <int NT>
 __global__ void __launch_bounds__(kPrepThreads) gemv_i8_prep_kernel(const PrepParams P) {
+  // x, M and the workspace may still be in use by the kernel before this one
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // let the dependent gemv grid launch now; it waits for this grid before reading our output
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ __align__(16) uint8_t smem[];
@@ -379,6 +381,9 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
     asm volatile("cp.async.wait_group 0;\n" ::: "memory");
   }
   __syncthreads();
+  // the scratch has been read: the next call's prep kernel may launch (it waits for this grid
+  // to finish before it writes anything)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ---- 3. main loop
   float accf[2][NT][4];
@@ -531,18 +536,25 @@ G8Plan plan_gemv_i8(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, i
   p.nt = ntok <= 1 ? 1 : ntok <= 2 ? 2 : 4;
   p.nchunk = (int)((L + 511) / 512);
   const int sms = sm_count();
-  // about 10 chunks (40 KB of fragments per token pair) per slice
+  auto smem_of = [&](int sc) {
+    return (size_t)p.nt * sc * g8::kFragBytesPerChunk +
+           (size_t)g8::kWarps * g8::kMaxPairsPerWarp * g8::kSlotFloatsPerNT * p.nt * 4 +
+           (size_t)sc * p.nt * 8 * 4;
+  };
+  // a warp's run must touch at most kMaxPairsPerWarp pairs: ceil(npair/16) + 1 <= 3
+  auto pairs_ok = [&](int R) {
+    const int npair = ((N + R - 1) / R + 31) / 32;
+    return (npair + g8::kWarps - 1) / g8::kWarps + 1 <= g8::kMaxPairsPerWarp;
+  };
+  // about 10 chunks (40 KB of fragments per token pair) per slice: whole rows per CTA would
+  // drop the cross-slice sums but costs more, every CTA then copying all fragments
   const int sc0 = std::max(1, 10 / p.nt);
   p.S = (p.nchunk + sc0 - 1) / sc0;
   p.sc = (p.nchunk + p.S - 1) / p.S;
   p.R = std::max(1, std::min(sms / std::min(p.S, sms), (N + 31) / 32));
   p.nctas = p.S * p.R;
-  // a warp's run must touch at most kMaxPairsPerWarp pairs: ceil(npair/16) + 1 <= 3
-  const int npair = ((N + p.R - 1) / p.R + 31) / 32;
-  if ((npair + g8::kWarps - 1) / g8::kWarps + 1 > g8::kMaxPairsPerWarp) p.ok = false;
-  p.smem = (size_t)p.nt * p.sc * g8::kFragBytesPerChunk +
-           (size_t)g8::kWarps * g8::kMaxPairsPerWarp * g8::kSlotFloatsPerNT * p.nt * 4 +
-           (size_t)p.sc * p.nt * 8 * 4;
+  if (!pairs_ok(p.R)) p.ok = false;
+  p.smem = smem_of(p.sc);
   const int span = (512 / D + 2) * d;
   p.xs_floats = Bh > 0 ? ((span + Bh - 1) / Bh + 1) * Bh : span;
   p.prep_smem = ((size_t)batch * p.xs_floats + (size_t)batch * 576 + 1024) * 4;
@@ -561,19 +573,23 @@ static cudaError_t launch_nt(const G8Plan& pl, const PrepParams& Q, const G8Para
   if (e != cudaSuccess) return e;
   e = ensure_smem((const void*)gemv_i8_kernel<NT>, pl.smem, smem_set);
   if (e != cudaSuccess) return e;
-  gemv_i8_prep_kernel<NT><<<pl.nchunk, kPrepThreads, pl.prep_smem, st>>>(Q);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(pl.nctas);
-  cfg.blockDim = dim3(g8::kThreads);
-  cfg.dynamicSmemBytes = pl.smem;
-  cfg.stream = st;
+  // both kernels use programmatic dependent launch: each waits for its predecessor's results
+  // (griddepcontrol.wait) before it reads them, so only the launch latency overlaps
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.nchunk);
+  cfg.blockDim = dim3(kPrepThreads);
+  cfg.dynamicSmemBytes = pl.prep_smem;
+  cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gemv_i8_prep_kernel<NT>, Q);
+  if (e != cudaSuccess) return e;
+  cfg.gridDim = dim3(pl.nctas);
+  cfg.blockDim = dim3(g8::kThreads);
+  cfg.dynamicSmemBytes = pl.smem;
   e = cudaLaunchKernelEx(&cfg, gemv_i8_kernel<NT>, P);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

@@ -167,6 +167,15 @@ LQ_API lq_status lq_gemm_noalloc(const void* x, lq_dtype xdt, int32_t batch,
  * failure) and clear it. Returns LQ_OK, or the lq_status that the word records. */
 LQ_API lq_status lq_device_status(void* workspace, int32_t* code, lq_stream stream);
 
+/* Checks the device-side timeout path: launches one warp that waits on a barrier nothing ever
+ * arrives on, with the bounded wait the kernels use (suspending try_wait plus a %globaltimer
+ * deadline) cut to limit_ms (1..1000). When the deadline passes the warp records
+ * LQ_ETIMEOUT in the workspace status word and returns; lq_device_status then reports it.
+ * The context stays usable: the same workspace serves the next lq_gemm once the status has
+ * been read. No counterpart on the pages. Errors: LQ_EINVAL (null or misaligned workspace,
+ * limit out of range), LQ_ECUDA (launch). */
+LQ_API lq_status lq_check_wait_timeout(void* workspace, int32_t limit_ms, lq_stream stream);
+
 /* Static text for a status code. */
 LQ_API const char* lq_status_string(lq_status status);
 

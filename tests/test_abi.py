@@ -64,6 +64,13 @@ def _r256(n):
     return -(-n // 256) * 256
 
 
+def test_wait_timeout_check_arguments_without_gpu(L):
+    assert L.lq_check_wait_timeout(None, 20, None) == lq.LQ_EINVAL
+    assert "workspace" in L.lq_last_error().decode()
+    assert L.lq_check_wait_timeout(ctypes.c_void_p(256), 0, None) == lq.LQ_EINVAL
+    assert "limit_ms" in L.lq_last_error().decode()
+
+
 def test_gemm_launches(L):
     assert lq.gemm_launches(1, 4096, 4096, 10, 24, 256) == 2        # int8 GEMV
     assert lq.gemm_launches(2048, 8192, 28672, 10, 24, 256) == 2    # tcgen05 GEMM
