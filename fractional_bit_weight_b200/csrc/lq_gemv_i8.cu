@@ -32,6 +32,7 @@ namespace g8 {
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
 constexpr int kFragBytesPerChunk = 16 * 32 * 8;  // 16 MMAs (2 k-halves x 8 bit positions)
+constexpr int kHalfBytesPerChunk = kFragBytesPerChunk / 2;   // one token: lanes 0-15 or 16-31
 constexpr int kMaxTokens = 8;
 constexpr int kPrefetch = 4;                      // items of stored bits in flight per warp
 constexpr int kMaxPairsPerWarp = 3;               // fp32 partial slots per warp
@@ -51,7 +52,7 @@ struct PrepParams {
   int nchunk;
   int sc;               // chunks per slice (fragments are stored slice by slice)
   int xs_floats;        // whitening scratch per token
-  uint2* frags;         // [S][NT][sc][16][32]
+  uint2* frags;         // [S][2*NT token halves][sc][16][16]
   float* wtab;          // [nchunk][NT][8]
   float* csum;          // [nchunk][batch]
 };
@@ -72,7 +73,8 @@ struct G8Params {
   int nchunk;           // 512-bit chunks per row
   int sc;               // chunks per slice
   int S;                // slices
-  int R;                // row ranges
+  int R;                // row ranges: range i has rq + (i < rrem) rows
+  int rq, rrem;         // N / R and N % R
 };
 
 __device__ __forceinline__ void imma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -115,13 +117,36 @@ __device__ __forceinline__ void planes4(float a, int (&P)[4]) {
   P[3] = __float2int_rn(r);
 }
 
+// v[r] = x[i0 + min(r, E - 1)] as fp32 for r < 8, all eight loads issued before the first use
+__device__ __forceinline__ void load8_as_f32(const void* p, int dt, int64_t i0, int E,
+                                             float (&v)[8]) {
+  if (dt == LQ_BF16) {
+    const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(p) + i0;
+    __nv_bfloat16 h[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) h[r] = q[min(r, E - 1)];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) v[r] = __bfloat162float(h[r]);
+  } else if (dt == LQ_F16) {
+    const __half* q = static_cast<const __half*>(p) + i0;
+    __half h[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) h[r] = q[min(r, E - 1)];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) v[r] = __half2float(h[r]);
+  } else {
+    const float* q = static_cast<const float*>(p) + i0;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) v[r] = q[min(r, E - 1)];
+  }
+}
+
 constexpr int kPrepThreads = 512;
+static_assert(kPrepThreads == 512, "the prep reductions assume 16 warps");
 
 // One CTA per chunk; see the file comment.
 template <int NT>
 __global__ void __launch_bounds__(kPrepThreads) gemv_i8_prep_kernel(const PrepParams P) {
-  // x, M and the workspace may still be in use by the kernel before this one
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   // let the dependent gemv grid launch now; it waits for this grid before reading our output
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ __align__(16) uint8_t smem[];
@@ -134,10 +159,10 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_i8_prep_kernel(const PrepPa
 
   const int c = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t q0 = (int64_t)c * 512;
-  const int64_t q1 = min(q0 + 512, P.L);
-  const int nq = (int)(q1 - q0);
-  const int g_lo = (int)(q0 / P.D), g_hi = (int)((q1 - 1) / P.D);
+  const int q0 = c * 512;                       // the plan keeps L below 2^30
+  const int q1 = min(q0 + 512, (int)P.L);
+  const int nq = q1 - q0;
+  const int g_lo = q0 / P.D, g_hi = (q1 - 1) / P.D;
   const int k0 = g_lo * P.d;
   const int k1 = min((g_hi + 1) * P.d, P.K);
   const int Bh = P.T.block;
@@ -147,23 +172,30 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_i8_prep_kernel(const PrepPa
     base = blk0 * Bh;
     span = ((k1 + Bh - 1) / Bh - blk0) * Bh;
   }
-  for (int i = tid; i < P.d * P.D; i += kPrepThreads) Ms[i] = P.M[i];
+  // M: copied by the highest threads first, which the warp-level whitening below leaves idle
+  for (int i = kPrepThreads - 1 - tid; i < P.d * P.D; i += kPrepThreads) Ms[i] = P.M[i];
   // 1. whitened inputs of every token
   if (Bh >= 32 && Bh <= 256) {
     const int E = Bh >> 5;
     const int nblk = span / Bh;
     for (int task = warp; task < P.batch * nblk; task += kPrepThreads / 32) {
       const int tok = task / nblk, b = task - tok * nblk;
-      float v[8];
+      // all loads of the lane are issued before any is used (indices past E repeat the last
+      // element and are discarded), so the whole block costs one memory round trip
+      const int kl = base + b * Bh + E * lane;
+      float v[8], cs[8];
+      int8_t sg[8];
+      load8_as_f32(P.x, P.xdt, (int64_t)tok * P.K + kl, E, v);
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
-        if (r < E) {
-          const int k = base + b * Bh + E * lane + r;
-          float a = load_as_f32(P.x, P.xdt, (int64_t)tok * P.K + k);
-          if (P.T.chan_scale) a *= P.T.chan_scale[k];
-          if (P.T.sign && P.T.sign[k] < 0) a = -a;
-          v[r] = a;
-        }
+        const int k = kl + min(r, E - 1);
+        cs[r] = P.T.chan_scale ? P.T.chan_scale[k] : 1.f;
+        sg[r] = P.T.sign ? P.T.sign[k] : (int8_t)1;
+      }
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        v[r] *= cs[r];
+        if (sg[r] < 0) v[r] = -v[r];
       }
 #pragma unroll
       for (int h = 1; h < 8; h <<= 1)
@@ -175,15 +207,16 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_i8_prep_kernel(const PrepPa
               v[r] = a + c2;
               v[r + h] = a - c2;
             }
+      // the lane stages run on all eight registers without a guard, so their shuffles
+      // overlap (registers past E hold copies and are never stored)
 #pragma unroll
       for (int m = 1; m < 32; m <<= 1) {
         const bool upper = (lane & m) != 0;
+        float o[8];
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
-          if (r < E) {
-            const float o = __shfl_xor_sync(0xffffffffu, v[r], m);
-            v[r] = upper ? o - v[r] : v[r] + o;
-          }
+        for (int r = 0; r < 8; ++r) o[r] = __shfl_xor_sync(0xffffffffu, v[r], m);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) v[r] = upper ? o[r] - v[r] : v[r] + o[r];
       }
       float* xt = xs + tok * P.xs_floats + b * Bh + E * lane;
 #pragma unroll
@@ -227,7 +260,7 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_i8_prep_kernel(const PrepPa
     const int e = tid;
     int gg = 0, jj = 0, dv = 0;
     if (e < nq) {
-      const int qi = (int)(q0 + e);
+      const int qi = q0 + e;
       gg = qi / P.D;
       jj = qi - gg * P.D;
       dv = min(P.d, P.K - gg * P.d);
@@ -238,8 +271,12 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_i8_prep_kernel(const PrepPa
       for (int ii = 0; ii < dv; ++ii) acc = fmaf(Ms[ii * P.D + jj], xg[ii], acc);
       acc *= P.T.inv_sqrt;
       zs[tok * kZP + e + 8 * (e >> 7)] = acc;
-      const float m = warp_max(fabsf(acc));
-      const float su = warp_sum(acc);
+      float m = fabsf(acc), su = acc;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        su += __shfl_xor_sync(0xffffffffu, su, o);
+      }
       if (lane == 0) {
         s_red[0][tok][warp] = m;
         s_red[1][tok][warp] = su;
@@ -247,41 +284,46 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_i8_prep_kernel(const PrepPa
     }
   }
   __syncthreads();
-  if (tid < P.batch) {
+  // warp w < 2*NT serves token slot w: the 16 warp maxima and sums reduced across lanes, the
+  // power-of-two scale S (|z| * S < 64), the chunk's sum of z and its four plane weights
+  if (warp < 2 * NT) {
+    const int tok = warp;
     float m = 0.f, su = 0.f;
-    for (int w = 0; w < kPrepThreads / 32; ++w) {
-      m = fmaxf(m, s_red[0][tid][w]);
-      su += s_red[1][tid][w];
+    if (tok < P.batch && lane < kPrepThreads / 32) {
+      m = s_red[0][tok][lane];
+      su = s_red[1][tok][lane];
+    }
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) {
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      su += __shfl_xor_sync(0xffffffffu, su, o);
     }
     int ex = 0;
     frexpf(m, &ex);                                         // m = f * 2^ex, f in [0.5, 1)
-    const float S = m > 0.f ? ldexpf(1.f, 6 - ex) : 1.f;    // |z| * S < 64
-    s_scale[tid] = S;
-    P.csum[(int64_t)c * P.batch + tid] = su;
-  }
-  if (tid < NT * 8) {
-    const int nt = tid >> 3, col = tid & 7, tok = nt * 2 + (col >> 2), pl = col & 3;
-    float w = 0.f;
-    if (tok < P.batch) {
-      float m = 0.f;
-      for (int ww = 0; ww < kPrepThreads / 32; ++ww) m = fmaxf(m, s_red[0][tok][ww]);
-      int ex = 0;
-      frexpf(m, &ex);
-      w = -2.f / (m > 0.f ? ldexpf(1.f, 6 - ex) : 1.f);
-      for (int k = 0; k < pl; ++k) w *= (float)(1.0 / 254.0);
+    const float S = m > 0.f ? ldexpf(1.f, 6 - ex) : 1.f;
+    if (lane == 0 && tok < P.batch) {
+      s_scale[tok] = S;
+      P.csum[(int64_t)c * P.batch + tok] = su;
     }
-    P.wtab[(int64_t)c * NT * 8 + tid] = w;
+    if (lane < 4) {
+      float w = 0.f;
+      if (tok < P.batch) {
+        w = -2.f / S;
+        for (int k = 0; k < lane; ++k) w *= (float)(1.0 / 254.0);
+      }
+      P.wtab[(int64_t)c * NT * 8 + (tok >> 1) * 8 + (tok & 1) * 4 + lane] = w;
+    }
   }
   __syncthreads();
-  // 3. quantise and store: thread -> (token slot, tt, j, h, p); its 4 values e0 + 8*i fill one
-  // 32-bit word per plane, word (j*8 + p)*64 + 2*(4*col + tt) + h of the chunk's fragment block
+  // 3. quantise and store: thread -> (token, tt, j, h, p); its 4 values e0 + 8*i fill one
+  // 32-bit word per plane: register h of lane 4*plane + tt for MMA (j, p) in the token's half
+  // (only tokens < batch are stored; the GEMV gives absent tokens zero B registers)
   const int sl = c / P.sc, cl = c - sl * P.sc;
-  for (int gi = tid; gi < 2 * NT * 128; gi += kPrepThreads) {
+  for (int gi = tid; gi < P.batch * 128; gi += kPrepThreads) {
     const int tok = gi >> 7, grp = gi & 127;
     const int pl8 = grp & 7, tt = (grp >> 3) & 3, hl = (grp >> 5) & 1, jl = grp >> 6;
-    const int nt = tok >> 1, cb = (tok & 1) * 4;
     uint32_t w4[4] = {0u, 0u, 0u, 0u};
-    if (tok < P.batch) {
+    {
       const float Sp = s_scale[tok] * __int_as_float((127 - pl8) << 23);   // S * 2^-p, exact
       const int e0 = 128 * tt + 64 * jl + 32 * hl + pl8;
       const float* zc = zs + tok * kZP + e0 + 8 * tt;
@@ -293,10 +335,11 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_i8_prep_kernel(const PrepPa
         for (int pl = 0; pl < 4; ++pl) w4[pl] |= ((uint32_t)Pq[pl] & 0xffu) << (8 * i);
       }
     }
+    // token tok's half: the B-operand registers of lanes 16*(tok&1) .. +15 (lane 4*plane + tt)
     uint32_t* fw = reinterpret_cast<uint32_t*>(P.frags) +
-                   (((size_t)sl * NT + nt) * P.sc + cl) * (g8::kFragBytesPerChunk / 4);
+                   (((size_t)sl * 2 * NT + tok) * P.sc + cl) * (g8::kHalfBytesPerChunk / 4);
 #pragma unroll
-    for (int pl = 0; pl < 4; ++pl) fw[(jl * 8 + pl8) * 64 + 2 * (4 * (cb + pl) + tt) + hl] = w4[pl];
+    for (int pl = 0; pl < 4; ++pl) fw[((jl * 8 + pl8) * 16 + 4 * pl + tt) * 2 + hl] = w4[pl];
   }
 }
 
@@ -305,6 +348,7 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
   extern __shared__ __align__(16) uint8_t smem[];
   __shared__ float s_sumz[g8::kMaxTokens];
   __shared__ int s_pfirst[g8::kWarps];
+  __shared__ int s_wrange[2][g8::kWarps * g8::kMaxPairsPerWarp];
   __shared__ int s_last;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -312,18 +356,21 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
   const int sl = blockIdx.x % P.S, ri = blockIdx.x / P.S;
   const int c0 = sl * P.sc;
   const int nc = min(P.sc, P.nchunk - c0);
-  const int ra = (int)((int64_t)ri * P.N / P.R);
-  const int rb = (int)((int64_t)(ri + 1) * P.N / P.R);
-  const int npair = (rb - ra + 31) / 32;
+  // no divisions on the way to the first loads: row ranges from the host's N / R and N % R,
+  // warp runs by a shift (16 warps)
+  const int ra = ri * P.rq + min(ri, P.rrem);
+  const int rb = ra + P.rq + (ri < P.rrem ? 1 : 0);
+  const int npair = (rb - ra + 31) >> 5;
   const int items = npair * nc;
-  const int i0 = (int)((int64_t)warp * items / g8::kWarps);
-  const int i1 = (int)((int64_t)(warp + 1) * items / g8::kWarps);
+  static_assert(g8::kWarps == 16, "warp runs are computed with a shift by 4");
+  const int i0 = (warp * items) >> 4;
+  const int i1 = ((warp + 1) * items) >> 4;
   const int n = i1 - i0;
   const int pfirst = i0 / nc;
 
   constexpr int kSlotFloats = g8::kSlotFloatsPerNT * NT;
-  uint2* sfr = reinterpret_cast<uint2*>(smem);                                  // [NT][sc][16][32]
-  float* slots = reinterpret_cast<float*>(smem + (size_t)NT * P.sc * g8::kFragBytesPerChunk);
+  uint2* sfr = reinterpret_cast<uint2*>(smem);                        // [batch][sc][16][16]
+  float* slots = reinterpret_cast<float*>(smem + (size_t)P.batch * P.sc * g8::kHalfBytesPerChunk);
   float* wts = slots + (size_t)g8::kWarps * g8::kMaxPairsPerWarp * kSlotFloats; // [sc][NT][8]
 
   // ---- 1. start streaming: item i = (pair i / nc, chunk c0 + i % nc)
@@ -364,8 +411,10 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
   // ---- 2. this slice's fragments and column weights (written by the prep kernel)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   {
-    const int nvec = NT * P.sc * g8::kFragBytesPerChunk / 16;
-    const uint4* src = reinterpret_cast<const uint4*>(P.frags) + (size_t)sl * nvec;
+    // the halves of tokens 0 .. batch-1 are a contiguous prefix of the slice's block
+    const int nvec = P.batch * P.sc * g8::kHalfBytesPerChunk / 16;
+    const uint4* src = reinterpret_cast<const uint4*>(P.frags) +
+                       (size_t)sl * 2 * NT * P.sc * g8::kHalfBytesPerChunk / 16;
     uint4* dst = reinterpret_cast<uint4*>(sfr);
     for (int i = tid; i < nvec; i += g8::kThreads) {
       const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst + i);
@@ -373,17 +422,15 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
     }
     asm volatile("cp.async.commit_group;\n" ::: "memory");
     for (int i = tid; i < nc * NT * 8; i += g8::kThreads) wts[i] = P.wtab[(size_t)c0 * NT * 8 + i];
-    if (tid < P.batch) {
+    if (warp < P.batch) {   // warp t: this slice's sum of z of token t, one load per lane
       float a = 0.f;
-      for (int c = 0; c < nc; ++c) a += P.csum[(int64_t)(c0 + c) * P.batch + tid];
-      s_sumz[tid] = a;
+      for (int c = lane; c < nc; c += 32) a += P.csum[(int64_t)(c0 + c) * P.batch + warp];
+      a = warp_sum(a);
+      if (lane == 0) s_sumz[warp] = a;
     }
     asm volatile("cp.async.wait_group 0;\n" ::: "memory");
   }
   __syncthreads();
-  // the scratch has been read: the next call's prep kernel may launch (it waits for this grid
-  // to finish before it writes anything)
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ---- 3. main loop
   float accf[2][NT][4];
@@ -394,7 +441,8 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
       accf[a][nt][0] = accf[a][nt][1] = accf[a][nt][2] = accf[a][nt][3] = 0.f;
   int ppr = pfirst, pc = i0 - pfirst * nc;         // position of the next item to process
   bool phasB = ra + ppr * 32 + 16 < rb;
-  const uint2* fb = sfr + lane;
+  // this lane's B registers: token 2*nt + (lane >> 4), entry lane & 15 of that token's half
+  const uint2* fb = sfr + (size_t)(lane >> 4) * P.sc * 256 + (lane & 15);
   auto park = [&]() {
     float* sp = slots + ((size_t)(warp * g8::kMaxPairsPerWarp + (ppr - pfirst)) * 2 * 32 + lane) * 4 * NT;
 #pragma unroll
@@ -407,7 +455,7 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
       }
   };
   auto process = [&](const uint4 (&u)[4]) {
-    const uint2* fc = fb + (size_t)pc * 512;
+    const uint2* fc = fb + (size_t)pc * 256;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       int ac[2][2][4];   // [tile][k-half]: four independent accumulation chains
@@ -424,7 +472,9 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
           const uint32_t msk = 0x01010101u << p;
-          const uint2 bv = fc[((size_t)nt * P.sc * 16 + j * 8 + p) * 32];
+          const uint2 bv = 2 * nt + (lane >> 4) < P.batch
+                               ? fc[(size_t)nt * 2 * P.sc * 256 + (j * 8 + p) * 16]
+                               : make_uint2(0u, 0u);
           imma_u8s8(ac[0][j], a0 & msk, a1 & msk, a2 & msk, a3 & msk, bv.x, bv.y);
           if (phasB) imma_u8s8(ac[1][j], b0 & msk, b1 & msk, b2 & msk, b3 & msk, bv.x, bv.y);
         }
@@ -457,6 +507,18 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
     }
   }
   if (n > 0 && pc != 0) park();   // the run ended inside a pair
+  if (n == 0) {
+    // an empty run (fewer items than warps) can fall inside a pair's warp range: its first
+    // slot, the one the pair maps to, reads as zero
+    float* sp = slots + (size_t)warp * g8::kMaxPairsPerWarp * kSlotFloats;
+    for (int i = lane; i < kSlotFloats; i += 32) sp[i] = 0.f;
+  }
+  // warps whose runs overlap pair pr: first w with ((w+1)*items)>>4 > pr*nc, last w with
+  // (w*items)>>4 < (pr+1)*nc
+  for (int pr = tid; pr < npair; pr += g8::kThreads) {
+    s_wrange[0][pr] = (16 * (pr * nc + 1) + items - 1) / items - 1;
+    s_wrange[1][pr] = (16 * (pr + 1) * nc + items - 1) / items - 1;
+  }
   __syncthreads();
 
   // ---- 4. per (row, token): this slice's value = its sum of z + warps' partials in warp order
@@ -466,24 +528,20 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
     const int rr = e - tok * rows;
     const int pr = rr >> 5, a = (rr >> 4) & 1, r = rr & 15;
     const int nt = tok >> 1, cb = (tok & 1) * 4;
-    // warp w owns items [floor(w*items/16), floor((w+1)*items/16)); item i belongs to warp
-    // ceil(16*(i+1)/items) - 1
-    const int wlo = (int)(((int64_t)(pr * nc + 1) * g8::kWarps + items - 1) / items) - 1;
-    const int whi = (int)(((int64_t)((pr + 1) * nc) * g8::kWarps + items - 1) / items) - 1;
+    // the four plane columns of (row, token) in a parked C fragment
+    int off[4];
+#pragma unroll
+    for (int pl = 0; pl < 4; ++pl) {
+      const int col = cb + pl;
+      off[pl] = (4 * (r & 7) + (col >> 1)) * 4 * NT + nt * 4 + 2 * (r >> 3) + (col & 1);
+    }
+    const int wlo = s_wrange[0][pr], whi = s_wrange[1][pr];
     float v = 0.f;
-    for (int w = max(0, wlo); w <= min(g8::kWarps - 1, whi); ++w) {
-      const int wi0 = (int)((int64_t)w * items / g8::kWarps);
-      const int wi1 = (int)((int64_t)(w + 1) * items / g8::kWarps);
-      if (wi0 == wi1 || wi1 <= pr * nc || wi0 >= (pr + 1) * nc) continue;
+#pragma unroll 4
+    for (int w = wlo; w <= whi; ++w) {
       const float* sp =
           slots + ((size_t)(w * g8::kMaxPairsPerWarp + (pr - s_pfirst[w])) * 2 + a) * 32 * 4 * NT;
-#pragma unroll
-      for (int pl = 0; pl < 4; ++pl) {
-        const int col = cb + pl;
-        const int ln = 4 * (r & 7) + (col >> 1);
-        const int i = 2 * (r >> 3) + (col & 1);
-        v += sp[ln * 4 * NT + nt * 4 + i];
-      }
+      v += (sp[off[0]] + sp[off[1]]) + (sp[off[2]] + sp[off[3]]);
     }
     const int row = ra + rr;
     const float part = s_sumz[tok] + v;
@@ -494,20 +552,34 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
   }
   if (P.S == 1) return;
 
-  // ---- cross-slice completion by the last CTA of this row range
-  __threadfence();
+  // ---- cross-slice completion by the last CTA of this row range (one fence and one atomic,
+  // by thread 0, after the barrier that orders the CTA's partial stores before them)
   __syncthreads();
   uint32_t* ctr = P.counters + ri;
-  if (tid == 0) s_last = (atomicAdd(ctr, 1u) == (uint32_t)(P.S - 1));
+  if (tid == 0) {
+    __threadfence();
+    const bool last = atomicAdd(ctr, 1u) == (uint32_t)(P.S - 1);
+    if (last) __threadfence();
+    s_last = last;
+  }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   for (int e = tid; e < rows * P.batch; e += g8::kThreads) {
     const int tok = e / rows;
     const int row = ra + (e - tok * rows);
+    const float sv = load_as_f32(P.s, P.sdt, row);
+    const float* pp = P.partials + (int64_t)tok * P.N + row;
+    const int64_t stride = (int64_t)P.batch * P.N;
+    // slices added in slice order; eight loads in flight per step
     float a = 0.f;
-    for (int k = 0; k < P.S; ++k) a += __ldcg(&P.partials[((int64_t)k * P.batch + tok) * P.N + row]);
-    P.y[(int64_t)tok * P.N + row] = load_as_f32(P.s, P.sdt, row) * a;
+    for (int k0 = 0; k0 < P.S; k0 += 8) {
+      float pk[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) pk[j] = k0 + j < P.S ? __ldcg(pp + (k0 + j) * stride) : 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a += pk[j];
+    }
+    P.y[(int64_t)tok * P.N + row] = sv * a;
   }
   if (tid == 0) *ctr = 0u;   // ready for the next call on this workspace
 }
@@ -537,7 +609,7 @@ G8Plan plan_gemv_i8(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, i
   p.nchunk = (int)((L + 511) / 512);
   const int sms = sm_count();
   auto smem_of = [&](int sc) {
-    return (size_t)p.nt * sc * g8::kFragBytesPerChunk +
+    return (size_t)batch * sc * g8::kHalfBytesPerChunk +
            (size_t)g8::kWarps * g8::kMaxPairsPerWarp * g8::kSlotFloatsPerNT * p.nt * 4 +
            (size_t)sc * p.nt * 8 * 4;
   };
@@ -546,9 +618,9 @@ G8Plan plan_gemv_i8(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, i
     const int npair = ((N + R - 1) / R + 31) / 32;
     return (npair + g8::kWarps - 1) / g8::kWarps + 1 <= g8::kMaxPairsPerWarp;
   };
-  // about 10 chunks (40 KB of fragments per token pair) per slice: whole rows per CTA would
-  // drop the cross-slice sums but costs more, every CTA then copying all fragments
-  const int sc0 = std::max(1, 10 / p.nt);
+  // about 40 KB of fragments (20 chunks of one token) per slice: every CTA of a slice copies
+  // them from L2, which costs more than the cross-slice sums beyond that size
+  const int sc0 = std::max(1, 20 / batch);
   p.S = (p.nchunk + sc0 - 1) / sc0;
   p.sc = (p.nchunk + p.S - 1) / p.S;
   p.R = std::max(1, std::min(sms / std::min(p.S, sms), (N + 31) / 32));
@@ -573,23 +645,22 @@ static cudaError_t launch_nt(const G8Plan& pl, const PrepParams& Q, const G8Para
   if (e != cudaSuccess) return e;
   e = ensure_smem((const void*)gemv_i8_kernel<NT>, pl.smem, smem_set);
   if (e != cudaSuccess) return e;
-  // both kernels use programmatic dependent launch: each waits for its predecessor's results
-  // (griddepcontrol.wait) before it reads them, so only the launch latency overlaps
+  // the prep kernel is an ordinary launch (launched with programmatic dependence on the
+  // previous call's GEMV it measured slower); the GEMV is launched with programmatic dependence
+  // on the prep kernel, so its CTAs start streaming stored bits while the prep runs
+  gemv_i8_prep_kernel<NT><<<pl.nchunk, kPrepThreads, pl.prep_smem, st>>>(Q);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(pl.nchunk);
-  cfg.blockDim = dim3(kPrepThreads);
-  cfg.dynamicSmemBytes = pl.prep_smem;
-  cfg.stream = st;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, gemv_i8_prep_kernel<NT>, Q);
-  if (e != cudaSuccess) return e;
   cfg.gridDim = dim3(pl.nctas);
   cfg.blockDim = dim3(g8::kThreads);
   cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, gemv_i8_kernel<NT>, P);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -634,6 +705,8 @@ cudaError_t launch_gemv_i8(const G8Plan& pl, const void* x, int xdt, int32_t bat
   P.sc = pl.sc;
   P.S = pl.S;
   P.R = pl.R;
+  P.rq = N / pl.R;
+  P.rrem = N % pl.R;
   switch (pl.nt) {
     case 1: return launch_nt<1>(pl, Q, P, st);
     case 2: return launch_nt<2>(pl, Q, P, st);
