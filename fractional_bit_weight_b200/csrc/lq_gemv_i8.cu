@@ -77,13 +77,23 @@ struct G8Params {
   int rq, rrem;         // N / R and N % R
 };
 
+// d += A * B (no side effects: the compiler may schedule it freely)
 __device__ __forceinline__ void imma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                           uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};\n"
       : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// d = A * B, the first MMA of an accumulation chain (C = 0)
+__device__ __forceinline__ void imma_u8s8_first(int (&d)[4], uint32_t a0, uint32_t a1,
+                                                uint32_t a2, uint32_t a3, uint32_t b0,
+                                                uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%10,%10,%10,%10};\n"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
 }
 
 __device__ __forceinline__ uint4 ldg_stream_v4(const uint8_t* p) {
@@ -370,14 +380,14 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
 
   constexpr int kSlotFloats = g8::kSlotFloatsPerNT * NT;
   uint2* sfr = reinterpret_cast<uint2*>(smem);                        // [batch][sc][16][16]
-  float* slots = reinterpret_cast<float*>(smem + (size_t)P.batch * P.sc * g8::kHalfBytesPerChunk);
+  uint2* zblk = sfr + (size_t)P.batch * P.sc * 256;                   // [16][16] zeros
+  float* slots = reinterpret_cast<float*>(zblk + 256);
   float* wts = slots + (size_t)g8::kWarps * g8::kMaxPairsPerWarp * kSlotFloats; // [sc][NT][8]
 
   // ---- 1. start streaming: item i = (pair i / nc, chunk c0 + i % nc)
   const int64_t last_off = P.row_bytes - 16;
   int lpr = pfirst, lc = i0 - pfirst * nc;       // position of the next item to load
   const uint8_t* rowp[4];
-  bool lhasB = false;
   auto set_rows = [&](int pr) {
     const int r = ra + pr * 32 + g;
 #pragma unroll
@@ -385,17 +395,15 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
       const int row = r + 8 * k;
       rowp[k] = P.packed + (int64_t)(row < rb ? row : ra) * P.row_bytes + 16 * t;
     }
-    lhasB = ra + pr * 32 + 16 < rb;
   };
   auto load_next = [&](uint4 (&u)[4]) {
     int64_t off = (int64_t)(c0 + lc) * 64;
     off = off + 16 * t > last_off ? last_off - 16 * t : off;   // last chunk: stay in the row
+    // rows past the range read row ra; their sums are computed but never stored
     u[0] = ldg_stream_v4(rowp[0] + off);
     u[1] = ldg_stream_v4(rowp[1] + off);
-    if (lhasB) {
-      u[2] = ldg_stream_v4(rowp[2] + off);
-      u[3] = ldg_stream_v4(rowp[3] + off);
-    }
+    u[2] = ldg_stream_v4(rowp[2] + off);
+    u[3] = ldg_stream_v4(rowp[3] + off);
     if (++lc == nc) {
       lc = 0;
       if (++lpr < npair) set_rows(lpr);
@@ -421,6 +429,7 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src + i) : "memory");
     }
     asm volatile("cp.async.commit_group;\n" ::: "memory");
+    if (tid < 128) reinterpret_cast<uint4*>(zblk)[tid] = make_uint4(0u, 0u, 0u, 0u);
     for (int i = tid; i < nc * NT * 8; i += g8::kThreads) wts[i] = P.wtab[(size_t)c0 * NT * 8 + i];
     if (warp < P.batch) {   // warp t: this slice's sum of z of token t, one load per lane
       float a = 0.f;
@@ -440,9 +449,16 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
     for (int nt = 0; nt < NT; ++nt)
       accf[a][nt][0] = accf[a][nt][1] = accf[a][nt][2] = accf[a][nt][3] = 0.f;
   int ppr = pfirst, pc = i0 - pfirst * nc;         // position of the next item to process
-  bool phasB = ra + ppr * 32 + 16 < rb;
-  // this lane's B registers: token 2*nt + (lane >> 4), entry lane & 15 of that token's half
-  const uint2* fb = sfr + (size_t)(lane >> 4) * P.sc * 256 + (lane & 15);
+  // this lane's B registers in tile nt: token 2*nt + (lane >> 4), entry lane & 15 of that
+  // token's half; a token past the batch reads the zero block at every chunk
+  const uint2* fbase[NT];
+  int fstride[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int tk = 2 * nt + (lane >> 4);
+    fbase[nt] = (tk < P.batch ? sfr + (size_t)tk * P.sc * 256 : zblk) + (lane & 15);
+    fstride[nt] = tk < P.batch ? 256 : 0;
+  }
   auto park = [&]() {
     float* sp = slots + ((size_t)(warp * g8::kMaxPairsPerWarp + (ppr - pfirst)) * 2 * 32 + lane) * 4 * NT;
 #pragma unroll
@@ -455,37 +471,42 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
       }
   };
   auto process = [&](const uint4 (&u)[4]) {
-    const uint2* fc = fb + (size_t)pc * 256;
+    // one accumulation chain per (tile nt, 16-row half a); the masked A registers of each
+    // (k-half j, bit p) are shared by all tiles
+    int ac[NT][2][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      int ac[2][2][4];   // [tile][k-half]: four independent accumulation chains
+    for (int j = 0; j < 2; ++j) {
+      const uint32_t a0 = j ? u[0].z : u[0].x, a2 = j ? u[0].w : u[0].y;
+      const uint32_t a1 = j ? u[1].z : u[1].x, a3 = j ? u[1].w : u[1].y;
+      const uint32_t b0 = j ? u[2].z : u[2].x, b2 = j ? u[2].w : u[2].y;
+      const uint32_t b1 = j ? u[3].z : u[3].x, b3 = j ? u[3].w : u[3].y;
 #pragma unroll
-      for (int a = 0; a < 2; ++a)
+      for (int p = 0; p < 8; ++p) {
+        const uint32_t msk = 0x01010101u << p;
+        const uint32_t m0 = a0 & msk, m1 = a1 & msk, m2 = a2 & msk, m3 = a3 & msk;
+        const uint32_t n0 = b0 & msk, n1 = b1 & msk, n2 = b2 & msk, n3 = b3 & msk;
 #pragma unroll
-        for (int j = 0; j < 2; ++j) ac[a][j][0] = ac[a][j][1] = ac[a][j][2] = ac[a][j][3] = 0;
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const uint32_t a0 = j ? u[0].z : u[0].x, a2 = j ? u[0].w : u[0].y;
-        const uint32_t a1 = j ? u[1].z : u[1].x, a3 = j ? u[1].w : u[1].y;
-        const uint32_t b0 = j ? u[2].z : u[2].x, b2 = j ? u[2].w : u[2].y;
-        const uint32_t b1 = j ? u[3].z : u[3].x, b3 = j ? u[3].w : u[3].y;
-#pragma unroll
-        for (int p = 0; p < 8; ++p) {
-          const uint32_t msk = 0x01010101u << p;
-          const uint2 bv = 2 * nt + (lane >> 4) < P.batch
-                               ? fc[(size_t)nt * 2 * P.sc * 256 + (j * 8 + p) * 16]
-                               : make_uint2(0u, 0u);
-          imma_u8s8(ac[0][j], a0 & msk, a1 & msk, a2 & msk, a3 & msk, bv.x, bv.y);
-          if (phasB) imma_u8s8(ac[1][j], b0 & msk, b1 & msk, b2 & msk, b3 & msk, bv.x, bv.y);
+        for (int nt = 0; nt < NT; ++nt) {
+          const uint2 bv = fbase[nt][pc * fstride[nt] + (j * 8 + p) * 16];
+          if (j == 0 && p == 0) {
+            imma_u8s8_first(ac[nt][0], m0, m1, m2, m3, bv.x, bv.y);
+            imma_u8s8_first(ac[nt][1], n0, n1, n2, n3, bv.x, bv.y);
+          } else {
+            imma_u8s8(ac[nt][0], m0, m1, m2, m3, bv.x, bv.y);
+            imma_u8s8(ac[nt][1], n0, n1, n2, n3, bv.x, bv.y);
+          }
         }
       }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
       const float2 w = *reinterpret_cast<const float2*>(wts + (pc * NT + nt) * 8 + 2 * t);
 #pragma unroll
       for (int a = 0; a < 2; ++a) {
-        accf[a][nt][0] = fmaf((float)(ac[a][0][0] + ac[a][1][0]), w.x, accf[a][nt][0]);
-        accf[a][nt][1] = fmaf((float)(ac[a][0][1] + ac[a][1][1]), w.y, accf[a][nt][1]);
-        accf[a][nt][2] = fmaf((float)(ac[a][0][2] + ac[a][1][2]), w.x, accf[a][nt][2]);
-        accf[a][nt][3] = fmaf((float)(ac[a][0][3] + ac[a][1][3]), w.y, accf[a][nt][3]);
+        accf[a][nt][0] = fmaf((float)ac[nt][a][0], w.x, accf[a][nt][0]);
+        accf[a][nt][1] = fmaf((float)ac[nt][a][1], w.y, accf[a][nt][1]);
+        accf[a][nt][2] = fmaf((float)ac[nt][a][2], w.x, accf[a][nt][2]);
+        accf[a][nt][3] = fmaf((float)ac[nt][a][3], w.y, accf[a][nt][3]);
       }
     }
     // end of this pair's chunks: park the pair's partial in the warp's slot
@@ -493,7 +514,6 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
       pc = 0;
       park();
       ++ppr;
-      phasB = ra + ppr * 32 + 16 < rb;
     }
   };
 
@@ -609,7 +629,7 @@ G8Plan plan_gemv_i8(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, i
   p.nchunk = (int)((L + 511) / 512);
   const int sms = sm_count();
   auto smem_of = [&](int sc) {
-    return (size_t)batch * sc * g8::kHalfBytesPerChunk +
+    return (size_t)(batch * sc + 1) * g8::kHalfBytesPerChunk +
            (size_t)g8::kWarps * g8::kMaxPairsPerWarp * g8::kSlotFloatsPerNT * p.nt * 4 +
            (size_t)sc * p.nt * 8 * 4;
   };
