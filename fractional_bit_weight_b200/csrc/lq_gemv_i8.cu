@@ -10,9 +10,10 @@
 //  prep, one CTA per 512-bit chunk of the lifted dimension: whitens the Hadamard blocks that
 //    feed the chunk (a warp per block: the first butterfly stages in registers, the rest with
 //    lane shuffles), lifts them, z = M^T xt per block of d inputs, picks a power-of-two scale S
-//    from max|z| of the chunk, and splits z*S*2^-p, p = q mod 8, into four int8 planes (base
-//    254) stored in the register layout of the B operand of mma.m16n8k32 (8 columns = 2 tokens
-//    x 4 planes), with the chunk's column weights -2*254^-plane/S and its sum of z.
+//    from max|z| of the chunk, and splits z*S*2^-p, p = q mod 8, into three int8 planes (base
+//    254, ~23 bits, at least 16 of them kept at p = 7) stored in the register layout of the B
+//    operand of mma.m16n8k32 (8 columns = 2 tokens x 4 plane slots, the fourth slot empty),
+//    with the chunk's column weights -2*254^-plane/S and its sum of z.
 //  gemv, S slices of chunks x R row ranges, one CTA each (one per SM): starts streaming its
 //    stored bits into registers at once, waits for prep, copies its slice's fragments to shared
 //    memory, then runs the (32-row tile pair, chunk) items of its rows, pair-major, in 16 equal
@@ -31,8 +32,10 @@ namespace lq {
 namespace g8 {
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kFragBytesPerChunk = 16 * 32 * 8;  // 16 MMAs (2 k-halves x 8 bit positions)
-constexpr int kHalfBytesPerChunk = kFragBytesPerChunk / 2;   // one token: lanes 0-15 or 16-31
+constexpr int kPlanes = 3;                        // int8 planes per value (plane slot 3 empty)
+// one token's B registers for one chunk: the 12 lanes 16*(token&1) + 4*plane + tt, 16 MMAs
+constexpr int kTokLanes = 4 * kPlanes;
+constexpr int kTokBytesPerChunk = 16 * kTokLanes * 8;   // 1536
 constexpr int kMaxTokens = 8;
 constexpr int kPrefetch = 4;                      // items of stored bits in flight per warp
 constexpr int kMaxPairsPerWarp = 3;               // fp32 partial slots per warp
@@ -52,7 +55,7 @@ struct PrepParams {
   int nchunk;
   int sc;               // chunks per slice (fragments are stored slice by slice)
   int xs_floats;        // whitening scratch per token
-  uint2* frags;         // [S][2*NT token halves][sc][16][16]
+  uint2* frags;         // [S][2*NT tokens][sc][16 MMAs][12 lanes]
   float* wtab;          // [nchunk][NT][8]
   float* csum;          // [nchunk][batch]
 };
@@ -116,15 +119,13 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// four int8 planes of base 254: a ~= P0 + P1/254 + P2/254^2 + P3/254^3 (|a| < 64)
-__device__ __forceinline__ void planes4(float a, int (&P)[4]) {
+// three int8 planes of base 254: a ~= P0 + P1/254 + P2/254^2 (|a| < 64)
+__device__ __forceinline__ void planes3(float a, int (&P)[3]) {
   P[0] = __float2int_rn(a);
   float r = (a - (float)P[0]) * 254.f;
   P[1] = __float2int_rn(r);
   r = (r - (float)P[1]) * 254.f;
   P[2] = __float2int_rn(r);
-  r = (r - (float)P[2]) * 254.f;
-  P[3] = __float2int_rn(r);
 }
 
 // v[r] = x[i0 + min(r, E - 1)] as fp32 for r < 8, all eight loads issued before the first use
@@ -295,7 +296,8 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_i8_prep_kernel(const PrepPa
   }
   __syncthreads();
   // warp w < 2*NT serves token slot w: the 16 warp maxima and sums reduced across lanes, the
-  // power-of-two scale S (|z| * S < 64), the chunk's sum of z and its four plane weights
+  // power-of-two scale S (|z| * S < 64), the chunk's sum of z and its plane weights (the
+  // empty fourth slot gets 0)
   if (warp < 2 * NT) {
     const int tok = warp;
     float m = 0.f, su = 0.f;
@@ -317,7 +319,7 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_i8_prep_kernel(const PrepPa
     }
     if (lane < 4) {
       float w = 0.f;
-      if (tok < P.batch) {
+      if (tok < P.batch && lane < g8::kPlanes) {
         w = -2.f / S;
         for (int k = 0; k < lane; ++k) w *= (float)(1.0 / 254.0);
       }
@@ -332,24 +334,25 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_i8_prep_kernel(const PrepPa
   for (int gi = tid; gi < P.batch * 128; gi += kPrepThreads) {
     const int tok = gi >> 7, grp = gi & 127;
     const int pl8 = grp & 7, tt = (grp >> 3) & 3, hl = (grp >> 5) & 1, jl = grp >> 6;
-    uint32_t w4[4] = {0u, 0u, 0u, 0u};
+    uint32_t w4[g8::kPlanes] = {};
     {
       const float Sp = s_scale[tok] * __int_as_float((127 - pl8) << 23);   // S * 2^-p, exact
       const int e0 = 128 * tt + 64 * jl + 32 * hl + pl8;
       const float* zc = zs + tok * kZP + e0 + 8 * tt;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        int Pq[4];
-        planes4(zc[8 * i] * Sp, Pq);
+        int Pq[g8::kPlanes];
+        planes3(zc[8 * i] * Sp, Pq);
 #pragma unroll
-        for (int pl = 0; pl < 4; ++pl) w4[pl] |= ((uint32_t)Pq[pl] & 0xffu) << (8 * i);
+        for (int pl = 0; pl < g8::kPlanes; ++pl) w4[pl] |= ((uint32_t)Pq[pl] & 0xffu) << (8 * i);
       }
     }
-    // token tok's half: the B-operand registers of lanes 16*(tok&1) .. +15 (lane 4*plane + tt)
+    // token tok's block: register hl of lane 4*plane + tt (of the token's half) for MMA (j, p)
     uint32_t* fw = reinterpret_cast<uint32_t*>(P.frags) +
-                   (((size_t)sl * 2 * NT + tok) * P.sc + cl) * (g8::kHalfBytesPerChunk / 4);
+                   (((size_t)sl * 2 * NT + tok) * P.sc + cl) * (g8::kTokBytesPerChunk / 4);
 #pragma unroll
-    for (int pl = 0; pl < 4; ++pl) fw[((jl * 8 + pl8) * 16 + 4 * pl + tt) * 2 + hl] = w4[pl];
+    for (int pl = 0; pl < g8::kPlanes; ++pl)
+      fw[((jl * 8 + pl8) * g8::kTokLanes + 4 * pl + tt) * 2 + hl] = w4[pl];
   }
 }
 
@@ -379,8 +382,9 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
   const int pfirst = i0 / nc;
 
   constexpr int kSlotFloats = g8::kSlotFloatsPerNT * NT;
-  uint2* sfr = reinterpret_cast<uint2*>(smem);                        // [batch][sc][16][16]
-  uint2* zblk = sfr + (size_t)P.batch * P.sc * 256;                   // [16][16] zeros
+  constexpr int kTokU2 = g8::kTokBytesPerChunk / 8;                   // uint2 per token-chunk
+  uint2* sfr = reinterpret_cast<uint2*>(smem);                        // [batch][sc][16][12]
+  uint2* zblk = sfr + (size_t)P.batch * P.sc * kTokU2;                // 256 zeros
   float* slots = reinterpret_cast<float*>(zblk + 256);
   float* wts = slots + (size_t)g8::kWarps * g8::kMaxPairsPerWarp * kSlotFloats; // [sc][NT][8]
 
@@ -415,14 +419,18 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
   for (int k = 0; k < g8::kPrefetch; ++k)
     if (k < n) load_next(q[k]);
   if (lane == 0) s_pfirst[warp] = pfirst;
+  // the row scale of this thread's first output (element e = tid: row ra + tid % rows), loaded
+  // now so that the epilogue does not wait for it
+  const int rows = rb - ra;
+  const float sv0 = tid < rows * P.batch ? load_as_f32(P.s, P.sdt, ra + tid % rows) : 0.f;
 
   // ---- 2. this slice's fragments and column weights (written by the prep kernel)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   {
-    // the halves of tokens 0 .. batch-1 are a contiguous prefix of the slice's block
-    const int nvec = P.batch * P.sc * g8::kHalfBytesPerChunk / 16;
+    // the blocks of tokens 0 .. batch-1 are a contiguous prefix of the slice's fragments
+    const int nvec = P.batch * P.sc * g8::kTokBytesPerChunk / 16;
     const uint4* src = reinterpret_cast<const uint4*>(P.frags) +
-                       (size_t)sl * 2 * NT * P.sc * g8::kHalfBytesPerChunk / 16;
+                       (size_t)sl * 2 * NT * P.sc * g8::kTokBytesPerChunk / 16;
     uint4* dst = reinterpret_cast<uint4*>(sfr);
     for (int i = tid; i < nvec; i += g8::kThreads) {
       const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst + i);
@@ -456,8 +464,9 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int tk = 2 * nt + (lane >> 4);
-    fbase[nt] = (tk < P.batch ? sfr + (size_t)tk * P.sc * 256 : zblk) + (lane & 15);
-    fstride[nt] = tk < P.batch ? 256 : 0;
+    const bool live = tk < P.batch && (lane & 15) < g8::kTokLanes;
+    fbase[nt] = (live ? sfr + (size_t)tk * P.sc * kTokU2 : zblk) + (lane & 15);
+    fstride[nt] = live ? kTokU2 : 0;
   }
   auto park = [&]() {
     float* sp = slots + ((size_t)(warp * g8::kMaxPairsPerWarp + (ppr - pfirst)) * 2 * 32 + lane) * 4 * NT;
@@ -487,7 +496,7 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
         const uint32_t n0 = b0 & msk, n1 = b1 & msk, n2 = b2 & msk, n3 = b3 & msk;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          const uint2 bv = fbase[nt][pc * fstride[nt] + (j * 8 + p) * 16];
+          const uint2 bv = fbase[nt][pc * fstride[nt] + (j * 8 + p) * g8::kTokLanes];
           if (j == 0 && p == 0) {
             imma_u8s8_first(ac[nt][0], m0, m1, m2, m3, bv.x, bv.y);
             imma_u8s8_first(ac[nt][1], n0, n1, n2, n3, bv.x, bv.y);
@@ -542,7 +551,6 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
   __syncthreads();
 
   // ---- 4. per (row, token): this slice's value = its sum of z + warps' partials in warp order
-  const int rows = rb - ra;
   for (int e = tid; e < rows * P.batch; e += g8::kThreads) {
     const int tok = e / rows;
     const int rr = e - tok * rows;
@@ -566,7 +574,7 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
     const int row = ra + rr;
     const float part = s_sumz[tok] + v;
     if (P.S == 1)
-      P.y[(int64_t)tok * P.N + row] = load_as_f32(P.s, P.sdt, row) * part;
+      P.y[(int64_t)tok * P.N + row] = (e == tid ? sv0 : load_as_f32(P.s, P.sdt, row)) * part;
     else
       P.partials[((int64_t)sl * P.batch + tok) * P.N + row] = part;
   }
@@ -587,7 +595,7 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
   for (int e = tid; e < rows * P.batch; e += g8::kThreads) {
     const int tok = e / rows;
     const int row = ra + (e - tok * rows);
-    const float sv = load_as_f32(P.s, P.sdt, row);
+    const float sv = e == tid ? sv0 : load_as_f32(P.s, P.sdt, row);
     const float* pp = P.partials + (int64_t)tok * P.N + row;
     const int64_t stride = (int64_t)P.batch * P.N;
     // slices added in slice order; eight loads in flight per step
@@ -629,7 +637,7 @@ G8Plan plan_gemv_i8(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, i
   p.nchunk = (int)((L + 511) / 512);
   const int sms = sm_count();
   auto smem_of = [&](int sc) {
-    return (size_t)(batch * sc + 1) * g8::kHalfBytesPerChunk +
+    return (size_t)batch * sc * g8::kTokBytesPerChunk + 256 * 8 +
            (size_t)g8::kWarps * g8::kMaxPairsPerWarp * g8::kSlotFloatsPerNT * p.nt * 4 +
            (size_t)sc * p.nt * 8 * 4;
   };
@@ -638,7 +646,7 @@ G8Plan plan_gemv_i8(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, i
     const int npair = ((N + R - 1) / R + 31) / 32;
     return (npair + g8::kWarps - 1) / g8::kWarps + 1 <= g8::kMaxPairsPerWarp;
   };
-  // about 40 KB of fragments (20 chunks of one token) per slice: every CTA of a slice copies
+  // about 30 KB of fragments (20 chunks of one token) per slice: every CTA of a slice copies
   // them from L2, which costs more than the cross-slice sums beyond that size
   const int sc0 = std::max(1, 20 / batch);
   p.S = (p.nchunk + sc0 - 1) / sc0;
@@ -650,7 +658,7 @@ G8Plan plan_gemv_i8(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, i
   const int span = (512 / D + 2) * d;
   p.xs_floats = Bh > 0 ? ((span + Bh - 1) / Bh + 1) * Bh : span;
   p.prep_smem = ((size_t)batch * p.xs_floats + (size_t)batch * 576 + 1024) * 4;
-  p.frag_bytes = (size_t)p.S * p.nt * p.sc * g8::kFragBytesPerChunk;
+  p.frag_bytes = (size_t)p.S * 2 * p.nt * p.sc * g8::kTokBytesPerChunk;
   p.wtab_bytes = (size_t)p.nchunk * p.nt * 8 * 4;
   p.csum_bytes = (size_t)p.nchunk * batch * 4;
   p.ok = p.ok && p.smem <= 220 * 1024 && p.prep_smem <= 200 * 1024;
