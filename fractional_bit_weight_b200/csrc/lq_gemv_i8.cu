@@ -39,6 +39,10 @@ constexpr int kTokBytesPerChunk = 16 * kTokLanes * 8;   // 1536
 constexpr int kMaxTokens = 8;
 constexpr int kPrefetch = 4;                      // items of stored bits in flight per warp
 constexpr int kMaxPairsPerWarp = 3;               // fp32 partial slots per warp
+// With four token tiles (5..8 tokens) the slots and registers are four times larger: two slots
+// per warp keep shared memory under the limit, two items in flight keep the registers in check.
+__host__ __device__ constexpr int max_pairs(int nt) { return nt >= 4 ? 2 : kMaxPairsPerWarp; }
+__host__ __device__ constexpr int prefetch(int nt) { return nt >= 4 ? 2 : kPrefetch; }
 constexpr int kSlotFloatsPerNT = 2 * 32 * 4;      // one tile pair: 2 tiles x 32 lanes x 4 regs
 }  // namespace g8
 
@@ -386,7 +390,8 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
   uint2* sfr = reinterpret_cast<uint2*>(smem);                        // [batch][sc][16][12]
   uint2* zblk = sfr + (size_t)P.batch * P.sc * kTokU2;                // 256 zeros
   float* slots = reinterpret_cast<float*>(zblk + 256);
-  float* wts = slots + (size_t)g8::kWarps * g8::kMaxPairsPerWarp * kSlotFloats; // [sc][NT][8]
+  constexpr int kMP = g8::max_pairs(NT), kPF = g8::prefetch(NT);
+  float* wts = slots + (size_t)g8::kWarps * kMP * kSlotFloats;                  // [sc][NT][8]
 
   // ---- 1. start streaming: item i = (pair i / nc, chunk c0 + i % nc)
   const int64_t last_off = P.row_bytes - 16;
@@ -414,9 +419,9 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
     }
   };
   if (n > 0) set_rows(lpr);
-  uint4 q[g8::kPrefetch][4];
+  uint4 q[kPF][4];
 #pragma unroll
-  for (int k = 0; k < g8::kPrefetch; ++k)
+  for (int k = 0; k < kPF; ++k)
     if (k < n) load_next(q[k]);
   if (lane == 0) s_pfirst[warp] = pfirst;
   // the row scale of this thread's first output (element e = tid: row ra + tid % rows), loaded
@@ -469,7 +474,7 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
     fstride[nt] = live ? kTokU2 : 0;
   }
   auto park = [&]() {
-    float* sp = slots + ((size_t)(warp * g8::kMaxPairsPerWarp + (ppr - pfirst)) * 2 * 32 + lane) * 4 * NT;
+    float* sp = slots + ((size_t)(warp * kMP + (ppr - pfirst)) * 2 * 32 + lane) * 4 * NT;
 #pragma unroll
     for (int a = 0; a < 2; ++a)
 #pragma unroll
@@ -526,12 +531,12 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
     }
   };
 
-  for (int kb = 0; kb < n; kb += g8::kPrefetch) {
+  for (int kb = 0; kb < n; kb += kPF) {
 #pragma unroll
-    for (int k = 0; k < g8::kPrefetch; ++k) {
+    for (int k = 0; k < kPF; ++k) {
       if (kb + k < n) {
         process(q[k]);
-        if (kb + k + g8::kPrefetch < n) load_next(q[k]);
+        if (kb + k + kPF < n) load_next(q[k]);
       }
     }
   }
@@ -539,7 +544,7 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
   if (n == 0) {
     // an empty run (fewer items than warps) can fall inside a pair's warp range: its first
     // slot, the one the pair maps to, reads as zero
-    float* sp = slots + (size_t)warp * g8::kMaxPairsPerWarp * kSlotFloats;
+    float* sp = slots + (size_t)warp * kMP * kSlotFloats;
     for (int i = lane; i < kSlotFloats; i += 32) sp[i] = 0.f;
   }
   // warps whose runs overlap pair pr: first w with ((w+1)*items)>>4 > pr*nc, last w with
@@ -568,7 +573,7 @@ __global__ void __launch_bounds__(g8::kThreads, 1) gemv_i8_kernel(const G8Params
 #pragma unroll 4
     for (int w = wlo; w <= whi; ++w) {
       const float* sp =
-          slots + ((size_t)(w * g8::kMaxPairsPerWarp + (pr - s_pfirst[w])) * 2 + a) * 32 * 4 * NT;
+          slots + ((size_t)(w * kMP + (pr - s_pfirst[w])) * 2 + a) * 32 * 4 * NT;
       v += (sp[off[0]] + sp[off[1]]) + (sp[off[2]] + sp[off[3]]);
     }
     const int row = ra + rr;
@@ -638,22 +643,33 @@ G8Plan plan_gemv_i8(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, i
   const int sms = sm_count();
   auto smem_of = [&](int sc) {
     return (size_t)batch * sc * g8::kTokBytesPerChunk + 256 * 8 +
-           (size_t)g8::kWarps * g8::kMaxPairsPerWarp * g8::kSlotFloatsPerNT * p.nt * 4 +
+           (size_t)g8::kWarps * g8::max_pairs(p.nt) * g8::kSlotFloatsPerNT * p.nt * 4 +
            (size_t)sc * p.nt * 8 * 4;
   };
-  // a warp's run must touch at most kMaxPairsPerWarp pairs: ceil(npair/16) + 1 <= 3
+  // a warp's run must touch at most max_pairs(nt) pairs: ceil(npair/16) + 1 <= max_pairs(nt)
   auto pairs_ok = [&](int R) {
     const int npair = ((N + R - 1) / R + 31) / 32;
-    return (npair + g8::kWarps - 1) / g8::kWarps + 1 <= g8::kMaxPairsPerWarp;
+    return (npair + g8::kWarps - 1) / g8::kWarps + 1 <= g8::max_pairs(p.nt);
   };
-  // about 30 KB of fragments (20 chunks of one token) per slice: every CTA of a slice copies
-  // them from L2, which costs more than the cross-slice sums beyond that size
-  const int sc0 = std::max(1, 20 / batch);
-  p.S = (p.nchunk + sc0 - 1) / sc0;
-  p.sc = (p.nchunk + p.S - 1) / p.S;
-  p.R = std::max(1, std::min(sms / std::min(p.S, sms), (N + 31) / 32));
+  // Slices of about 30 KB of fragments (20 chunks of one token): every CTA of a slice copies
+  // them from L2, which costs more than the cross-slice sums beyond that size. Where that
+  // leaves more rows per CTA than the warps' partial slots hold, the slices widen (fewer
+  // slices, so more row ranges) until the rows fit or the fragments outgrow shared memory.
+  p.ok = false;
+  for (int sc = std::min(std::max(1, 20 / batch), p.nchunk); sc <= p.nchunk; ++sc) {
+    const int S = (p.nchunk + sc - 1) / sc;
+    const int R = std::max(1, std::min(sms / std::min(S, sms), (N + 31) / 32));
+    const int scs = (p.nchunk + S - 1) / S;
+    if (smem_of(scs) > 220 * 1024) break;
+    if (!pairs_ok(R)) continue;
+    p.S = S;
+    p.sc = scs;
+    p.R = R;
+    p.ok = true;
+    break;
+  }
+  if (!p.ok) return p;
   p.nctas = p.S * p.R;
-  if (!pairs_ok(p.R)) p.ok = false;
   p.smem = smem_of(p.sc);
   const int span = (512 / D + 2) * d;
   p.xs_floats = Bh > 0 ? ((span + Bh - 1) / Bh + 1) * Bh : span;

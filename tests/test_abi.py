@@ -80,6 +80,16 @@ def test_gemm_launches(L):
     assert lq.gemm_launches(1, 4096, 4096, 10, 24, 3) == 0
 
 
+@pytest.mark.parametrize("K,N,max_single", [(4096, 4096, 8), (8192, 8192, 8), (8192, 28672, 4),
+                                            (28672, 8192, 4), (256, 128, 8), (40, 64, 8)])
+def test_small_batches_run_as_one_gemv(L, K, N, max_single):
+    """Up to 4 tokens on the Llama-3-70B MLP shapes, up to 8 on 4096- and 8192-wide layers, the
+    int8 GEMV runs once (prep + contraction): the slices widen until a CTA's rows fit its warps'
+    partial slots instead of splitting the batch into token groups."""
+    for b in range(1, max_single + 1):
+        assert lq.gemm_launches(b, K, N, 10, 24, 256) == 2, b
+
+
 @pytest.mark.parametrize("batch,K,N,d,D", [(64, 8192, 28672, 10, 24), (2048, 8192, 28672, 10, 24),
                                            (200, 512, 600, 10, 24), (300, 96, 513, 16, 32)])
 def test_workspace_of_tensor_core_path(L, batch, K, N, d, D):

@@ -46,11 +46,17 @@ def test_noalloc_matches_gemm_twice(K, N, d, D, batch):
 
 def test_noalloc_rejects_what_does_not_fit():
     fake = ctypes.c_void_p(0x10000)     # never dereferenced: the call is rejected first
-    # 8 tokens of a 2^20-input row: the slice partials alone need about 80 MB
-    rc = lq.lib().lq_gemm_noalloc(fake, lq.LQ_BF16, 8, None, fake, fake, fake, lq.LQ_F16, 10, 24,
-                                  1 << 20, 1024, fake, None)
+    # 1 token of a 2^24-input row: ~3900 K-slices, whose fragments and partials need far more
+    # than the library's scratch
+    rc = lq.lib().lq_gemm_noalloc(fake, lq.LQ_BF16, 1, None, fake, fake, fake, lq.LQ_F16, 10, 24,
+                                  1 << 24, 1024, fake, None)
     assert rc == lq.LQ_EINVAL
     assert "scratch" in lq.lib().lq_last_error().decode()
+    # 8 tokens of a 2^20-input row: no GEMV plan (the fragments of a slice wide enough for the
+    # rows to fit the partial slots outgrow shared memory)
+    rc = lq.lib().lq_gemm_noalloc(fake, lq.LQ_BF16, 8, None, fake, fake, fake, lq.LQ_F16, 10, 24,
+                                  1 << 20, 1024, fake, None)
+    assert rc in (lq.LQ_EINVAL, lq.LQ_EUNSUPPORTED)
     rc = lq.lib().lq_gemm_noalloc(fake, lq.LQ_BF16, 9, None, fake, fake, fake, lq.LQ_F16, 10, 24,
                                   4096, 4096, fake, None)
     assert rc == lq.LQ_EINVAL
