@@ -330,7 +330,8 @@ constexpr int kLiftChunk = 4096;   // lifted coordinates per pass of the prologu
 // One CTA per token: zh[t][0 .. Lp) fp16 (word-interleaved order, zero beyond L) and
 // inv_scale[t] = 2^-e. Dynamic shared memory: M in rows of D4 = D rounded up to 4 columns
 // (zero beyond D), xt zero-padded to Kp, then one pass of natural-order z.
-__global__ void __launch_bounds__(512)
+// four CTAs per SM (53 KB of shared memory each at K = 8192): a register cap of 32
+__global__ void __launch_bounds__(512, 4)
     lift_f16_kernel(const void* __restrict__ x, int xdt, int K, Whiten T,
                     const float* __restrict__ M, int d, int D, int Kp, int64_t L, int Lp,
                     __half* __restrict__ zh, float* __restrict__ inv_scale) {
@@ -347,7 +348,11 @@ __global__ void __launch_bounds__(512)
     const int i = k / D4, j = k - i * D4;
     sM[k] = j < D ? M[i * D + j] : 0.f;
   }
-  if (T.block > 0) {
+  if (T.block >= 32 && T.block <= 256) {
+    // a warp per Hadamard block, no barrier between the butterfly stages
+    for (int b = tid >> 5; b < K / T.block; b += blockDim.x >> 5)
+      warp_whiten_block(x, xdt, row, b * T.block, T.block >> 5, T, T.inv_sqrt, sx + b * T.block);
+  } else if (T.block > 0) {
     whiten_blocks_smem(x, xdt, row, K, T, 0, K / T.block, sx);   // ends with a barrier
   } else {
     for (int k = tid; k < K; k += blockDim.x) sx[k] = load_as_f32(x, xdt, row + k);

@@ -132,30 +132,6 @@ __device__ __forceinline__ void planes3(float a, int (&P)[3]) {
   P[2] = __float2int_rn(r);
 }
 
-// v[r] = x[i0 + min(r, E - 1)] as fp32 for r < 8, all eight loads issued before the first use
-__device__ __forceinline__ void load8_as_f32(const void* p, int dt, int64_t i0, int E,
-                                             float (&v)[8]) {
-  if (dt == LQ_BF16) {
-    const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(p) + i0;
-    __nv_bfloat16 h[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) h[r] = q[min(r, E - 1)];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) v[r] = __bfloat162float(h[r]);
-  } else if (dt == LQ_F16) {
-    const __half* q = static_cast<const __half*>(p) + i0;
-    __half h[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) h[r] = q[min(r, E - 1)];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) v[r] = __half2float(h[r]);
-  } else {
-    const float* q = static_cast<const float*>(p) + i0;
-#pragma unroll
-    for (int r = 0; r < 8; ++r) v[r] = q[min(r, E - 1)];
-  }
-}
-
 constexpr int kPrepThreads = 512;
 static_assert(kPrepThreads == 512, "the prep reductions assume 16 warps");
 
@@ -195,48 +171,8 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_i8_prep_kernel(const PrepPa
     const int nblk = span / Bh;
     for (int task = warp; task < P.batch * nblk; task += kPrepThreads / 32) {
       const int tok = task / nblk, b = task - tok * nblk;
-      // all loads of the lane are issued before any is used (indices past E repeat the last
-      // element and are discarded), so the whole block costs one memory round trip
-      const int kl = base + b * Bh + E * lane;
-      float v[8], cs[8];
-      int8_t sg[8];
-      load8_as_f32(P.x, P.xdt, (int64_t)tok * P.K + kl, E, v);
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const int k = kl + min(r, E - 1);
-        cs[r] = P.T.chan_scale ? P.T.chan_scale[k] : 1.f;
-        sg[r] = P.T.sign ? P.T.sign[k] : (int8_t)1;
-      }
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        v[r] *= cs[r];
-        if (sg[r] < 0) v[r] = -v[r];
-      }
-#pragma unroll
-      for (int h = 1; h < 8; h <<= 1)
-        if (h < E)
-#pragma unroll
-          for (int r = 0; r < 8; ++r)
-            if (r < E && (r & h) == 0) {
-              const float a = v[r], c2 = v[r + h];
-              v[r] = a + c2;
-              v[r + h] = a - c2;
-            }
-      // the lane stages run on all eight registers without a guard, so their shuffles
-      // overlap (registers past E hold copies and are never stored)
-#pragma unroll
-      for (int m = 1; m < 32; m <<= 1) {
-        const bool upper = (lane & m) != 0;
-        float o[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) o[r] = __shfl_xor_sync(0xffffffffu, v[r], m);
-#pragma unroll
-        for (int r = 0; r < 8; ++r) v[r] = upper ? o[r] - v[r] : v[r] + o[r];
-      }
-      float* xt = xs + tok * P.xs_floats + b * Bh + E * lane;
-#pragma unroll
-      for (int r = 0; r < 8; ++r)
-        if (r < E) xt[r] = v[r];
+      warp_whiten_block(P.x, P.xdt, (int64_t)tok * P.K, base + b * Bh, E, P.T, 1.f,
+                        xs + tok * P.xs_floats + b * Bh);
     }
     __syncthreads();
   } else {
