@@ -45,6 +45,10 @@ def _load(path=None):
     lib.orc_forward_lifted.restype = ctypes.c_int
     lib.orc_encode_bruteforce.argtypes = [_dp, _dp, i32, i32, _i8p]
     lib.orc_encode_bruteforce.restype = i64
+    lib.orc_encode_seeded.argtypes = [_dp, _dp, i32, i32, _i8p, _dp]
+    lib.orc_encode_seeded.restype = i64
+    lib.orc_encode_rows.argtypes = [_dp, i64, i32, _dp, i32, i32, i32, _i8p, _dp, ctypes.c_int]
+    lib.orc_encode_rows.restype = ctypes.c_int
     lib.orc_max_threads.argtypes = []
     lib.orc_max_threads.restype = ctypes.c_int
     return lib
@@ -197,6 +201,37 @@ def encode_bruteforce(w, M, d, D, _lib=None):
     if c < 0:
         raise ValueError("oracle encode rejected its arguments")
     return out, int(c)
+
+
+def encode_seeded(w, M, d, D, _lib=None):
+    """Seeded search (first d coordinates solved, the other D - d enumerated); returns
+    (b int8[D], index f, squared distance)."""
+    L = _lib or lib()
+    wf = _f64(w).reshape(d)
+    Mf = _f64(M).reshape(d, D)
+    out = np.zeros(D, dtype=np.int8)
+    dist = ctypes.c_double(0.0)
+    f = L.orc_encode_seeded(_ptr(wf, _dp), _ptr(Mf, _dp), d, D, _ptr(out, _i8p), ctypes.byref(dist))
+    if f < 0:
+        raise ValueError("oracle seeded encode rejected its arguments")
+    return out, int(f), float(dist.value)
+
+
+def encode_rows(w, M, d, D, mode, nthreads=0, _lib=None):
+    """Encodes w [N][K] block by block: (b int8 [N][G][D], err float64 [N][G]).
+    mode 0: exhaustive 2^D search; mode 1: seeded 2^(D-d) search."""
+    L = _lib or lib()
+    wf = _f64(w)
+    N, K = wf.shape
+    G = -(-K // d)
+    Mf = _f64(M).reshape(d, D)
+    b = np.zeros((N, G, D), dtype=np.int8)
+    err = np.zeros((N, G), dtype=np.float64)
+    rc = L.orc_encode_rows(_ptr(wf, _dp), N, K, _ptr(Mf, _dp), d, D, mode, _ptr(b, _i8p),
+                           _ptr(err, _dp), nthreads)
+    if rc != 0:
+        raise ValueError("oracle encode_rows rejected its arguments")
+    return b, err
 
 
 def max_threads(_lib=None):

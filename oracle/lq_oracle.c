@@ -309,6 +309,128 @@ int64_t orc_encode_bruteforce(const double* w, const double* M, int32_t d, int32
   return best;
 }
 
+/* Squared distance || w - M b ||^2 of the block w (length d) to the codeword b (length D). */
+static double orc_block_dist(const double* w, const double* M, int32_t d, int32_t D,
+                             const int8_t* b) {
+  double dist = 0.0;
+  for (int32_t i = 0; i < d; ++i) {
+    double r = w[i];
+    for (int32_t j = 0; j < D; ++j) r -= M[i * D + j] * (double)b[j];
+    dist += r * r;
+  }
+  return dist;
+}
+
+/* Seeded search, the review's "pseudo-inverse initialisation" that cuts the 2^D search of
+ * Eq. (1) to 2^(D-d) (romaanj.github.io review, "Method"; the cap D - d <= 20 is in its
+ * "Limitations"). Reading (the pages give no more): the first d coordinates are solved, the
+ * other D - d are enumerated. For every f in [0, 2^(D-d)), b_{d+k} = -1 exactly when bit k of
+ * f is set; r = w - sum_{j>=d} M[:,j] b_j; u solves M_S u = r with M_S = M[:, 0..d) (Gaussian
+ * elimination with partial pivoting); b_i = +1 when u_i >= 0, else -1 (i < d). The candidate
+ * with the smallest || w - M b ||^2 wins, ties keeping the smallest f. Writes b_out [D] and the
+ * distance; returns f, or -1 for invalid sizes or a singular M_S. */
+int64_t orc_encode_seeded(const double* w, const double* M, int32_t d, int32_t D, int8_t* b_out,
+                          double* dist_out) {
+  if (d < 1 || D < d || D > 32 || D - d > 24) return -1;
+  const int32_t F = D - d;
+  double* A = (double*)malloc(sizeof(double) * (size_t)d * (size_t)(d + 1));
+  int8_t* b = (int8_t*)malloc((size_t)D);
+  if (!A || !b) {
+    free(A);
+    free(b);
+    return -1;
+  }
+  int64_t best = -1;
+  double best_dist = 0.0;
+  int singular = 0;
+  for (int64_t f = 0; f < ((int64_t)1 << F) && !singular; ++f) {
+    for (int32_t k = 0; k < F; ++k) b[d + k] = ((f >> k) & 1) ? (int8_t)-1 : (int8_t)1;
+    /* augmented system [M_S | r] */
+    for (int32_t i = 0; i < d; ++i) {
+      double r = w[i];
+      for (int32_t k = 0; k < F; ++k) r -= M[i * D + d + k] * (double)b[d + k];
+      for (int32_t c = 0; c < d; ++c) A[i * (d + 1) + c] = M[i * D + c];
+      A[i * (d + 1) + d] = r;
+    }
+    for (int32_t c = 0; c < d; ++c) {               /* forward elimination */
+      int32_t piv = c;
+      for (int32_t i = c + 1; i < d; ++i)
+        if (fabs(A[i * (d + 1) + c]) > fabs(A[piv * (d + 1) + c])) piv = i;
+      if (A[piv * (d + 1) + c] == 0.0) {
+        singular = 1;
+        break;
+      }
+      if (piv != c)
+        for (int32_t k = 0; k <= d; ++k) {
+          const double t = A[c * (d + 1) + k];
+          A[c * (d + 1) + k] = A[piv * (d + 1) + k];
+          A[piv * (d + 1) + k] = t;
+        }
+      for (int32_t i = c + 1; i < d; ++i) {
+        const double m = A[i * (d + 1) + c] / A[c * (d + 1) + c];
+        for (int32_t k = c; k <= d; ++k) A[i * (d + 1) + k] -= m * A[c * (d + 1) + k];
+      }
+    }
+    if (singular) break;
+    for (int32_t c = d - 1; c >= 0; --c) {          /* back substitution: u into column d */
+      double u = A[c * (d + 1) + d];
+      for (int32_t k = c + 1; k < d; ++k) u -= A[c * (d + 1) + k] * A[k * (d + 1) + d];
+      u /= A[c * (d + 1) + c];
+      A[c * (d + 1) + d] = u;
+      b[c] = u >= 0.0 ? (int8_t)1 : (int8_t)-1;
+    }
+    const double dist = orc_block_dist(w, M, d, D, b);
+    if (best < 0 || dist < best_dist) {
+      best = f;
+      best_dist = dist;
+      memcpy(b_out, b, (size_t)D);
+    }
+  }
+  free(A);
+  free(b);
+  if (singular) return -1;
+  if (dist_out) *dist_out = best_dist;
+  return best;
+}
+
+/* Encodes a weight matrix w [N][K] block by block (K zero-padded to G*d): b [N][G][D] in
+ * {+1,-1} and err [N][G] = || w_block - M b ||^2. mode 0: exhaustive search over all 2^D
+ * codewords; mode 1: the seeded search above. Blocks are independent; threads split rows.
+ * Returns 0, or -1 if a block was rejected. */
+int orc_encode_rows(const double* w, int64_t N, int32_t K, const double* M, int32_t d, int32_t D,
+                    int32_t mode, int8_t* b, double* err, int nthreads) {
+  if (N < 0 || K < 1 || d < 1 || D < d || D > 32 || (mode != 0 && mode != 1)) return -1;
+  if (mode == 0 && D > 24) return -1;
+  const int64_t G = orc_groups(K, d);
+  int failed = 0;
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(static) reduction(| : failed)
+#endif
+  for (int64_t n = 0; n < N; ++n) {
+    double blk[64];
+    for (int64_t g = 0; g < G; ++g) {
+      for (int32_t i = 0; i < d; ++i) {
+        const int64_t k = g * d + i;
+        blk[i] = k < K ? w[n * K + k] : 0.0;
+      }
+      int8_t* bo = b + (n * G + g) * D;
+      double dist = 0.0;
+      int64_t r;
+      if (mode == 0) {
+        r = orc_encode_bruteforce(blk, M, d, D, bo);
+        if (r >= 0) dist = orc_block_dist(blk, M, d, D, bo);
+      } else {
+        r = orc_encode_seeded(blk, M, d, D, bo, &dist);
+      }
+      if (r < 0) failed = 1;
+      if (err) err[n * G + g] = dist;
+    }
+  }
+  (void)nthreads;
+  return failed ? -1 : 0;
+}
+
 int orc_max_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

@@ -349,4 +349,73 @@ def pin_encoder(orc):
         assert np.allclose(M @ b, w0, atol=1e-12)
 
 
+def _all_codewords(D):
+    C = np.array(list(itertools.product([0, 1], repeat=D)))[:, ::-1]     # row c: bits of c
+    return 1 - 2 * C.astype(np.float64)                                   # [2^D][D], bit 1 -> -1
+
+
+def pin_encoder_seeded(orc):
+    """Seeded search (first d coordinates solved, the other D - d enumerated), checked against
+    numpy: its distance is the distance of its code, its free part is its index, its solved part
+    is the sign of numpy.linalg.solve, it never beats the exhaustive minimum, and it finds a
+    planted codeword exactly."""
+    rng = _rng(15)
+    for d, D in [(1, 1), (3, 3), (1, 2), (2, 5), (3, 8), (4, 10), (6, 12)]:
+        M = rng.standard_normal((d, D))
+        cw = _all_codewords(D)
+        for _ in range(5):
+            w = rng.standard_normal(d)
+            b, f, dist = orc.encode_seeded(w, M, d, D)
+            bf = b.astype(np.float64)
+            assert abs(dist - ((w - M @ bf) ** 2).sum()) <= 1e-12 * (1.0 + dist)
+            assert f == sum(1 << k for k in range(D - d) if b[d + k] < 0)
+            u = np.linalg.solve(M[:, :d], w - M[:, d:] @ bf[d:])
+            assert np.array_equal(b[:d], np.where(u >= 0, 1, -1).astype(np.int8))
+            best = ((w[None, :] - cw @ M.T) ** 2).sum(axis=1).min()
+            assert dist >= best - 1e-12
+            # the winner is the best of all 2^(D-d) candidates the reading defines
+            cand = []
+            for ff in range(1 << (D - d)):
+                bF = np.array([-1.0 if (ff >> k) & 1 else 1.0 for k in range(D - d)])
+                uu = np.linalg.solve(M[:, :d], w - M[:, d:] @ bF)
+                bb = np.concatenate([np.where(uu >= 0, 1.0, -1.0), bF])
+                cand.append(((w - M @ bb) ** 2).sum())
+            assert f == int(np.argmin(cand))
+        # a planted codeword is recovered (the candidate with its free part solves exactly)
+        c0 = int(rng.integers(0, 1 << D))
+        b, f, dist = orc.encode_seeded(M @ cw[c0], M, d, D)
+        assert np.array_equal(b, cw[c0].astype(np.int8)) and dist < 1e-20
+    # zero free columns: every free part ties, f = 0 wins, the rest is sign(M_S^-1 w)
+    d, D = 3, 6
+    M = np.concatenate([rng.standard_normal((d, d)), np.zeros((d, D - d))], axis=1)
+    w = rng.standard_normal(d)
+    b, f, _ = orc.encode_seeded(w, M, d, D)
+    assert f == 0 and np.array_equal(b[d:], np.ones(D - d, dtype=np.int8))
+    assert np.array_equal(b[:d], np.where(np.linalg.solve(M[:, :d], w) >= 0, 1, -1))
+
+
+def pin_encode_rows(orc):
+    """Whole-matrix encoding: K is zero-padded to a multiple of d, err is || w_blk - M b ||^2
+    (numpy), the exhaustive mode is numpy's argmin over all codewords, and the thread count
+    changes nothing."""
+    rng = _rng(16)
+    d, D, N, K = 3, 7, 5, 13                      # 13 = 4 full blocks + 1 padded block
+    M = rng.standard_normal((d, D))
+    w = rng.standard_normal((N, K))
+    wp = np.concatenate([w, np.zeros((N, 2))], axis=1).reshape(N, 5, d)
+    cw = _all_codewords(D)
+    b0, e0 = orc.encode_rows(w, M, d, D, 0)
+    b1, e1 = orc.encode_rows(w, M, d, D, 1)
+    assert b0.shape == (N, 5, D) and e1.shape == (N, 5)
+    for n in range(N):
+        for g in range(5):
+            dist = ((wp[n, g][None, :] - cw @ M.T) ** 2).sum(axis=1)
+            assert np.array_equal(b0[n, g], cw[int(np.argmin(dist))].astype(np.int8))
+            for b, e in ((b0, e0), (b1, e1)):
+                assert abs(e[n, g] - ((wp[n, g] - M @ b[n, g]) ** 2).sum()) < 1e-12
+            assert e1[n, g] >= e0[n, g] - 1e-12
+    b2, e2 = orc.encode_rows(w, M, d, D, 1, nthreads=3)
+    assert np.array_equal(b2, b1) and np.array_equal(e2, e1)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
