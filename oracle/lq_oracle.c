@@ -380,7 +380,7 @@ int64_t orc_encode_seeded(const double* w, const double* M, int32_t d, int32_t D
       b[c] = u >= 0.0 ? (int8_t)1 : (int8_t)-1;
     }
     const double dist = orc_block_dist(w, M, d, D, b);
-    if (best < 0 || dist < best_dist) {
+    if (dist < best_dist || best < 0) {
       best = f;
       best_dist = dist;
       memcpy(b_out, b, (size_t)D);

@@ -43,6 +43,11 @@ MUTANTS = [
      "b[n * bits + q] = bit ? (int8_t)1 : (int8_t)-1;"),
     ("row_padding_8_bytes", "return (bytes + 15) / 16 * 16;", "return (bytes + 7) / 8 * 8;"),
     ("encoder_argmax", "if (best < 0 || dist < best_dist) {", "if (best < 0 || dist > best_dist) {"),
+    ("seeded_argmax", "if (dist < best_dist || best < 0) {", "if (dist > best_dist || best < 0) {"),
+    ("seeded_solved_sign", "b[c] = u >= 0.0 ? (int8_t)1 : (int8_t)-1;",
+     "b[c] = u >= 0.0 ? (int8_t)-1 : (int8_t)1;"),
+    ("seeded_free_bit_order", "b[d + k] = ((f >> k) & 1) ? (int8_t)-1 : (int8_t)1;",
+     "b[d + k] = ((f >> (F - 1 - k)) & 1) ? (int8_t)-1 : (int8_t)1;"),
     ("encoder_codeword_sign", "r -= M[i * D + j] * (((c >> j) & 1) ? -1.0 : 1.0);",
      "r -= M[i * D + j] * (((c >> j) & 1) ? 1.0 : -1.0);"),
     ("lift_padding_reads_next_block", "double v = (k < K) ? xt[t * K + k] : 0.0;",
