@@ -44,7 +44,15 @@ WORKLOADS = {
     "llama3_70b_down_b1": (3, 3, "gemv"),
     "sweep_d10D24_b1": (4, 8, "gemv"),
     "prefill_b2048": (5, 0, "gemm"),
+    # encoder: 512 rows of the q_proj shape, seeded 2^(D-d) search per block
+    "encode_seeded_512x4096_d10D24": (None, None, "encode"),
 }
+
+# the encoder workload: (N, K, d, D, mode, seed); w ~ N(0, 1) stands for whitened weights,
+# M ~ N(0, 1/D)
+ENCODE = {"encode_seeded_512x4096_d10D24": (512, 4096, 10, 24, lq.LQ_ENCODE_SEEDED, 5)}
+# fp32 FMA rate of B200 from its unit counts and clock: 148 SMs x 128 lanes x 2 flop x 1.965 GHz
+FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def parse():
@@ -321,6 +329,8 @@ def main():
     args = parse()
     ws, rank, local = dist_setup()
     cfg, idx, kind = WORKLOADS[args.workload]
+    if kind == "encode":
+        return encode_main(args, ws, rank, local)
     spec = synth.workload_specs(cfg)[idx]
     if args.impl == "reference":
         return reference_arm(args, spec, kind, ws, rank)
@@ -381,6 +391,114 @@ def main():
             (wl.flops() * frac / dt / 1e12)
         out["cpu_baseline"] = {"value": cpu_val, "unit": unit, "cores": threads, "kind": "oracle",
                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(out))
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+def encode_inputs(name):
+    N, K, d, D, mode, seed = ENCODE[name]
+    rng = np.random.Generator(np.random.PCG64([seed, N, K]))
+    M = (rng.standard_normal((d, D)) / np.sqrt(D)).astype(np.float32)
+    w = rng.standard_normal((N, K)).astype(np.float32)
+    return N, K, d, D, mode, M, w
+
+
+def encode_oracle_sample(name, budget_s=10.0):
+    """The oracle's seeded search on the host cores over the first rows of the workload, sized
+    to about budget_s; returns (weights per second, sample description, threads)."""
+    import oracle
+    N, K, d, D, mode, M, w = encode_inputs(name)
+    threads = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    oracle.encode_rows(w[:1, :d * 64], M, d, D, mode, nthreads=threads)     # 64 blocks
+    per_block = max(time.perf_counter() - t0, 1e-6) / 64
+    G = -(-K // d)
+    nblk = int(max(threads, min(N * G, budget_s / per_block)))
+    rows, cols = max(1, nblk // G), min(K, nblk * d)
+    t0 = time.perf_counter()
+    oracle.encode_rows(w[:rows, :cols], M, d, D, mode, nthreads=threads)
+    dt = time.perf_counter() - t0
+    done = rows * cols
+    return done / dt, f"{rows} rows x {cols} inputs of {N} x {K}, fp64 oracle", threads
+
+
+def encode_main(args, ws, rank, local):
+    """One step = one lq_encode call over the whole matrix (weights resident in HBM)."""
+    name = args.workload
+    N, K, d, D, mode, M, w = encode_inputs(name)
+    G = -(-K // d)
+    cand = N * G * (1 << (D - d)) if mode == lq.LQ_ENCODE_SEEDED else N * G * (1 << D)
+    if args.impl == "reference":
+        if rank == 0:
+            v, sample, threads = encode_oracle_sample(name)
+            print(json.dumps({
+                "impl": "reference", "metric": "lq_encode_weights_per_s", "value": v,
+                "unit": "weights/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": N * K / v * 1e3, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": name, "N": N, "K": K, "d": d, "D": D, "mode": "seeded"},
+                "cpu_baseline": {"value": v, "unit": "weights/s", "cores": threads,
+                                 "kind": "oracle", "sample": sample},
+                "e2e": {"value": v, "unit": "weights/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}))
+        if ws > 1:
+            torch.distributed.destroy_process_group()
+        return
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wd, Md = torch.from_numpy(w).to(dev), torch.from_numpy(M).to(dev)
+    b = torch.empty((N, G, D), dtype=torch.int8, device=dev)
+    lib = lq.lib()
+
+    def step(i, wsrc=None):
+        rc = lib.lq_encode(wd.data_ptr() if wsrc is None else wsrc.data_ptr(), N, K,
+                           Md.data_ptr(), d, D, mode, b.data_ptr(), None,
+                           torch.cuda.current_stream().cuda_stream)
+        if rc != lq.LQ_OK:
+            raise RuntimeError(lib.lq_last_error().decode())
+
+    with ClockSampler(local) as clk:
+        secs = time_steps(step, args.steps, args.warmup, ws)
+    secs = max_over_ranks(secs, ws)
+    per_step = secs / args.steps
+    value = N * K * args.steps * ws / secs
+    # algorithmic work of the incremental walk: per candidate 2d flops for u, d for r_F, d for
+    # e and 2d for the distance (6d), against the fp32 FMA rate
+    achieved = cand * 6 * d / per_step / 1e12
+    out = {
+        "metric": "lq_encode_weights_per_s", "value": value, "unit": "weights/s",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded: w N(0,1), M N(0,1/D))",
+        "config": {"workload": name, "N": N, "K": K, "d": d, "D": D, "mode": "seeded",
+                   "candidates_per_step": cand, "parallelism": f"replicas x{ws}",
+                   "l2": f"w is {N * K * 4 / 1e6:.1f} MB; the search is ALU-bound"},
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": FP32_TFLOPS,
+                     "unit": "TFLOP/s", "frac": achieved / FP32_TFLOPS, "traffic": None,
+                     "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 flop x 1.965 GHz"},
+        "gpu_launches": args.steps,
+        "timing": "CUDA events on the launching stream",
+        "clocks": clk.summary(),
+    }
+    if not args.no_e2e:
+        w_host = torch.from_numpy(w).pin_memory()
+        b_host = torch.empty((N, G, D), dtype=torch.int8).pin_memory()
+        w_dev = torch.empty_like(wd)
+
+        def e2e_step(i):
+            w_dev.copy_(w_host, non_blocking=True)
+            step(i, w_dev)
+            b_host.copy_(b, non_blocking=True)
+
+        e2e_secs = max_over_ranks(time_steps(e2e_step, args.steps, args.warmup, ws), ws)
+        out["e2e"] = {"value": N * K * args.steps * ws / e2e_secs, "unit": "weights/s",
+                      "h2d_bytes_per_step": N * K * 4, "d2h_bytes_per_step": N * G * D}
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        v, sample, threads = encode_oracle_sample(name)
+        out["cpu_baseline"] = {"value": v, "unit": "weights/s", "cores": threads,
+                               "kind": "oracle", "sample": sample}
     if rank == 0:
         print(json.dumps(out))
     if ws > 1:

@@ -27,7 +27,7 @@ LQ_OK, LQ_EINVAL, LQ_EUNSUPPORTED, LQ_ECUDA, LQ_ETIMEOUT, LQ_EDEVICE = range(6)
 LQ_F32, LQ_F16, LQ_BF16 = 0, 1, 2
 _DTYPES = {torch.float32: LQ_F32, torch.float16: LQ_F16, torch.bfloat16: LQ_BF16}
 
-EXPORTS = ("lq_abi_version", "lq_lifted_bits", "lq_row_stride_bytes", "lq_pack", "lq_unpack",
+EXPORTS = ("lq_abi_version", "lq_lifted_bits", "lq_row_stride_bytes", "lq_pack", "lq_unpack", "lq_encode",
            "lq_whiten", "lq_lift", "lq_gemm_workspace_bytes", "lq_gemm_launches", "lq_gemm",
            "lq_gemm_noalloc", "lq_check_wait_timeout",
            "lq_device_status", "lq_status_string", "lq_last_error")
@@ -55,6 +55,7 @@ def _declare(L):
         "lq_lifted_bits": ([i32, i32, i32], i64),
         "lq_row_stride_bytes": ([i32, i32, i32], i64),
         "lq_pack": ([vp, i32, i32, i32, i32, vp, vp], ctypes.c_int),
+        "lq_encode": ([vp, i32, i32, vp, i32, i32, i32, vp, vp, vp], ctypes.c_int),
         "lq_unpack": ([vp, i32, i32, i32, i32, vp, vp], ctypes.c_int),
         "lq_whiten": ([vp, ctypes.c_int, i32, i32, dp, vp, vp], ctypes.c_int),
         "lq_lift": ([vp, ctypes.c_int, i32, i32, dp, vp, i32, i32, vp, vp], ctypes.c_int),
@@ -146,6 +147,23 @@ def pack(b_pm1, K, d, D, out=None, stream=None):
     _check(lib().lq_pack(_dev(b_pm1, "b_pm1", (torch.int8,)), N, K, d, D,
                          _dev(out, "packed", (torch.int32,)), _stream(stream)), "lq_pack")
     return out
+
+
+LQ_ENCODE_EXACT, LQ_ENCODE_SEEDED = 0, 1
+
+
+def encode(w, M, d, D, mode=LQ_ENCODE_SEEDED, with_err=True, stream=None):
+    """Nearest-codeword codes of w [N][K] fp32 (see lq_encode): returns (b_pm1 int8
+    [N][ceil(K/d)][D], err fp32 [N][ceil(K/d)] or None). Pack b_pm1.view(N, -1) with pack()."""
+    N, K = w.shape
+    G = -(-K // d)
+    b = torch.empty((N, G, D), dtype=torch.int8, device=w.device)
+    err = torch.empty((N, G), dtype=torch.float32, device=w.device) if with_err else None
+    _check(lib().lq_encode(_dev(w, "w", (torch.float32,)), N, K, _dev(M, "M", (torch.float32,)),
+                           d, D, int(mode), _dev(b, "b_pm1", (torch.int8,)),
+                           _dev(err, "err", (torch.float32,)) if with_err else None,
+                           _stream(stream)), "lq_encode")
+    return b, err
 
 
 def unpack(packed, K, d, D, out=None, stream=None):

@@ -203,6 +203,26 @@ lq_status lq_pack(const int8_t* b_pm1, int32_t N, int32_t K, int32_t d, int32_t 
   return e == cudaSuccess ? LQ_OK : cuda_fail(e, "lq_pack");
 }
 
+lq_status lq_encode(const float* w, int32_t N, int32_t K, const float* M, int32_t d, int32_t D,
+                    int32_t mode, int8_t* b_pm1, float* err, lq_stream stream) {
+  clear_error();
+  if (!valid_code(K, d, D)) return fail(LQ_EINVAL, "invalid code sizes K=%d d=%d D=%d", K, d, D);
+  if (N < 0) return fail(LQ_EINVAL, "N = %d < 0", N);
+  if (mode != LQ_ENCODE_EXACT && mode != LQ_ENCODE_SEEDED)
+    return fail(LQ_EINVAL, "unknown encode mode %d", mode);
+  if (d > 16) return fail(LQ_EUNSUPPORTED, "lq_encode: d = %d > 16", d);
+  if (mode == LQ_ENCODE_EXACT && D > 24)
+    return fail(LQ_EUNSUPPORTED, "lq_encode: exact search with D = %d > 24", D);
+  if (mode == LQ_ENCODE_SEEDED && D - d > 24)
+    return fail(LQ_EUNSUPPORTED, "lq_encode: seeded search with D - d = %d > 24", D - d);
+  if (N == 0) return LQ_OK;
+  if (!w || !M || !b_pm1) return fail(LQ_EINVAL, "null pointer");
+  if (!aligned(w, 4) || !aligned(M, 4) || (err && !aligned(err, 4)))
+    return fail(LQ_EINVAL, "misaligned w/M/err");
+  cudaError_t e = lq::launch_encode(w, N, K, M, d, D, mode, b_pm1, err, (cudaStream_t)stream);
+  return e == cudaSuccess ? LQ_OK : cuda_fail(e, "lq_encode");
+}
+
 lq_status lq_unpack(const uint32_t* packed, int32_t N, int32_t K, int32_t d, int32_t D,
                     int8_t* b_pm1, lq_stream stream) {
   clear_error();

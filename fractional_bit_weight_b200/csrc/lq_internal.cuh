@@ -120,4 +120,9 @@ cudaError_t launch_gemm_tc(const TcPlan& pl, const void* x, int xdt, int32_t bat
                            const uint32_t* packed, int64_t row_bytes, int32_t N, const void* s,
                            int sdt, float* y, void* scratch, uint32_t* status, cudaStream_t st);
 
+// Nearest-codeword encoding, block by block: b [N][ceil(K/d)][D] +1/-1, err [N][G] or null.
+// mode 0: all 2^D codewords; mode 1: first d coordinates solved, the rest enumerated.
+cudaError_t launch_encode(const float* w, int64_t N, int32_t K, const float* M, int32_t d,
+                          int32_t D, int32_t mode, int8_t* b, float* err, cudaStream_t st);
+
 }  // namespace lq

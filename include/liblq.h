@@ -99,6 +99,34 @@ LQ_API lq_status lq_pack(const int8_t* b_pm1, int32_t N, int32_t K, int32_t d, i
 LQ_API lq_status lq_unpack(const uint32_t* packed, int32_t N, int32_t K, int32_t d, int32_t D,
                     int8_t* b_pm1, lq_stream stream);
 
+/* Encoding searches of lq_encode. */
+typedef enum lq_encode_mode {
+  LQ_ENCODE_EXACT = 0,   /* all 2^D codewords, D <= 24 */
+  LQ_ENCODE_SEEDED = 1   /* the first d coordinates solved, the other D - d enumerated */
+} lq_encode_mode;
+
+/* Nearest-codeword encoding of a weight matrix (paper sec. 3.1, the inner minimisation of
+ * Eq. (1): every length-d block w of a row becomes the b in {+1,-1}^D that minimises
+ * ||w - M b||^2; review "Method": the search in the lifted space, cut from 2^D to 2^(D-d)
+ * candidates by a pseudo-inverse initialisation, practical up to D - d = 20 by its
+ * "Limitations"). LQ_ENCODE_SEEDED reads that initialisation as: for every free part
+ * b_F in {+1,-1}^(D-d) (coordinates d..D-1), u = M_S^-1 (w - M_F b_F) with M_S = M[:, 0..d),
+ * b_i = +1 when u_i >= 0, else -1, for i < d. Either search keeps the candidate of smallest
+ * distance, ties going to the smallest index (the codeword c with b_j = -1 exactly when bit j
+ * of c is set, or the free part). Runs in fp32: candidates within fp32 rounding of each other
+ * may be ordered differently than in exact arithmetic.
+ *   w     [N][K] fp32 device, row-major; each row is zero-padded to ceil(K/d)*d.
+ *   M     [d][D] fp32 device.
+ *   b_pm1 [N][ceil(K/d)][D] int8 device, +1/-1: the codes in the layout lq_pack takes.
+ *   err   [N][ceil(K/d)] fp32 device or NULL: ||w_block - M b||^2 of every block; NaN for
+ *         LQ_ENCODE_SEEDED when M_S is singular.
+ * Errors: LQ_EINVAL for null pointers (w, M, b_pm1), misaligned w/M/err, N < 0, K < 1, d < 1,
+ * D < d, D > LQ_MAX_D or an unknown mode; LQ_EUNSUPPORTED for d > 16, exact with D > 24, or
+ * seeded with D - d > 24; LQ_ECUDA for a failed launch. N = 0 is a no-op. Asynchronous on
+ * `stream`. */
+LQ_API lq_status lq_encode(const float* w, int32_t N, int32_t K, const float* M, int32_t d,
+                           int32_t D, int32_t mode, int8_t* b_pm1, float* err, lq_stream stream);
+
 /* Whitening alone: xt = T(x) (review, "Method": Hadamard mixing plus scalings).
  *   x  [batch][K] of dtype xdt;  xt [batch][K] float32.
  * Errors: LQ_EINVAL (null pointers, batch < 0, K < 1, bad block), LQ_EUNSUPPORTED

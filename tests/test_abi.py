@@ -64,6 +64,22 @@ def _r256(n):
     return -(-n // 256) * 256
 
 
+def test_encode_arguments_without_gpu(L):
+    fake = ctypes.c_void_p(0x10000)     # never dereferenced: every call below returns first
+    S = None
+    assert L.lq_encode(None, 4, 16, fake, 2, 5, 1, fake, None, S) == lq.LQ_EINVAL
+    assert L.lq_encode(fake, 4, 16, fake, 2, 5, 7, fake, None, S) == lq.LQ_EINVAL    # mode
+    assert "mode" in L.lq_last_error().decode()
+    assert L.lq_encode(fake, 4, 16, fake, 5, 4, 1, fake, None, S) == lq.LQ_EINVAL    # D < d
+    assert L.lq_encode(fake, -1, 16, fake, 2, 5, 1, fake, None, S) == lq.LQ_EINVAL
+    assert L.lq_encode(ctypes.c_void_p(0x10002), 4, 16, fake, 2, 5, 1, fake, None, S) == \
+        lq.LQ_EINVAL                                                                  # w align
+    assert L.lq_encode(fake, 4, 64, fake, 17, 20, 1, fake, None, S) == lq.LQ_EUNSUPPORTED
+    assert L.lq_encode(fake, 4, 64, fake, 2, 25, 0, fake, None, S) == lq.LQ_EUNSUPPORTED
+    assert L.lq_encode(fake, 4, 64, fake, 2, 27, 1, fake, None, S) == lq.LQ_EUNSUPPORTED
+    assert L.lq_encode(fake, 0, 64, fake, 2, 5, 1, fake, None, S) == lq.LQ_OK        # no work
+
+
 def test_wait_timeout_check_arguments_without_gpu(L):
     assert L.lq_check_wait_timeout(None, 20, None) == lq.LQ_EINVAL
     assert "workspace" in L.lq_last_error().decode()
