@@ -49,6 +49,8 @@ def _load(path=None):
     lib.orc_encode_seeded.restype = i64
     lib.orc_encode_rows.argtypes = [_dp, i64, i32, _dp, i32, i32, i32, _i8p, _dp, ctypes.c_int]
     lib.orc_encode_rows.restype = ctypes.c_int
+    lib.orc_codebook_round.argtypes = [_dp, i64, _dp, i32, i32, i32, _i8p, ctypes.c_int]
+    lib.orc_codebook_round.restype = ctypes.c_double
     lib.orc_max_threads.argtypes = []
     lib.orc_max_threads.restype = ctypes.c_int
     return lib
@@ -232,6 +234,21 @@ def encode_rows(w, M, d, D, mode, nthreads=0, _lib=None):
     if rc != 0:
         raise ValueError("oracle encode_rows rejected its arguments")
     return b, err
+
+
+def codebook_round(w, M, d, D, mode=0, nthreads=0, _lib=None):
+    """One round of the codebook fit on samples w [S][d]: nearest codewords under M, then the
+    least-squares M. Returns (M_new [d][D], codes int8 [S][D], mse per weight before the
+    update)."""
+    L = _lib or lib()
+    wf = _f64(w).reshape(-1, d)
+    Mf = _f64(M).reshape(d, D).copy()
+    b = np.zeros((wf.shape[0], D), dtype=np.int8)
+    mse = L.orc_codebook_round(_ptr(wf, _dp), wf.shape[0], _ptr(Mf, _dp), d, D, mode,
+                               _ptr(b, _i8p), nthreads)
+    if mse < 0:
+        raise ValueError("oracle codebook_round rejected its arguments")
+    return Mf, b, float(mse)
 
 
 def max_threads(_lib=None):

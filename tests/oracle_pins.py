@@ -418,4 +418,47 @@ def pin_encode_rows(orc):
     assert np.array_equal(b2, b1) and np.array_equal(e2, e1)
 
 
+def pin_codebook_round(orc):
+    """One round of the codebook fit (nearest codewords, then least-squares M), checked against
+    numpy: the 1-bit scalar case in closed form (M = mean |w|), codes = numpy's argmin over all
+    codewords, the straight-through gradient sum (w - M b) b^T vanishing at the new M, exact
+    recovery of a codebook that generated the samples, order invariance, and a mean error that
+    never rises from round to round with the exhaustive search."""
+    rng = _rng(17)
+    # d = D = 1: b = sign(w) (ties to +1), M_new = mean |w|
+    w = rng.standard_normal((500, 1))
+    M1, b1, mse = orc.codebook_round(w, np.array([[0.3]]), 1, 1)
+    sg = np.where(w[:, 0] >= 0, 1, -1)
+    assert np.array_equal(b1[:, 0], sg)
+    assert abs(M1[0, 0] - np.abs(w).mean()) < 1e-12
+    assert abs(mse - ((w[:, 0] - 0.3 * sg) ** 2).mean()) < 1e-12
+    # (2, 5): codes are the exhaustive argmin; the new M zeroes the gradient
+    d, D = 2, 5
+    w = rng.standard_normal((300, d))
+    M0 = rng.standard_normal((d, D)) * 0.5
+    M1, b, mse = orc.codebook_round(w, M0, d, D)
+    cw = _all_codewords(D)
+    dist = ((w[:, None, :] - (cw @ M0.T)[None, :, :]) ** 2).sum(axis=2)
+    assert np.array_equal(b, cw[np.argmin(dist, axis=1)].astype(np.int8))
+    assert abs(mse - dist.min(axis=1).mean() / d) < 1e-12
+    bf = b.astype(np.float64)
+    grad = (w - bf @ M1.T).T @ bf
+    assert np.abs(grad).max() < 1e-9 * len(w)
+    # samples generated by a codebook are fitted exactly from that codebook
+    Mt = rng.standard_normal((d, D))
+    wt = _all_codewords(D) @ Mt.T
+    Mr, br, mr = orc.codebook_round(wt, Mt, d, D)
+    assert mr < 1e-24 and np.allclose(Mr, Mt, atol=1e-12)
+    # order of the samples does not matter
+    perm = rng.permutation(len(w))
+    Mp, _, msep = orc.codebook_round(w[perm], M0, d, D)
+    assert np.allclose(Mp, M1, atol=1e-12) and abs(msep - mse) < 1e-12
+    # exhaustive rounds never raise the mean error
+    M, last = M0, np.inf
+    for _ in range(5):
+        M, _, m = orc.codebook_round(w, M, d, D)
+        assert m <= last + 1e-12
+        last = m
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -48,6 +48,10 @@ MUTANTS = [
      "b[c] = u >= 0.0 ? (int8_t)-1 : (int8_t)1;"),
     ("seeded_free_bit_order", "b[d + k] = ((f >> k) & 1) ? (int8_t)-1 : (int8_t)1;",
      "b[d + k] = ((f >> (F - 1 - k)) & 1) ? (int8_t)-1 : (int8_t)1;"),
+    ("codebook_gram_transposed", "C[j * (D + d) + k] += (double)bn[j] * (double)bn[k];",
+     "C[j * (D + d) + k] += (double)bn[j] * (double)bn[j];"),
+    ("codebook_cross_term_sign", "A[i * D + j] += w[n * d + i] * (double)bn[j];",
+     "A[i * D + j] -= w[n * d + i] * (double)bn[j];"),
     ("encoder_codeword_sign", "r -= M[i * D + j] * (((c >> j) & 1) ? -1.0 : 1.0);",
      "r -= M[i * D + j] * (((c >> j) & 1) ? 1.0 : -1.0);"),
     ("lift_padding_reads_next_block", "double v = (k < K) ? xt[t * K + k] : 0.0;",
