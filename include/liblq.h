@@ -185,7 +185,10 @@ LQ_API lq_status lq_gemm(const void* x, lq_dtype xdt, int32_t batch, const lq_wh
  *   - Every call on a device shares the one array and leaves it ready for the next call; calls
  *     that overlap on the GPU (different streams, or threads without ordering) race on it and
  *     must be serialised by the caller.
- * Errors: as lq_gemm, plus LQ_EINVAL for batch > 8 or a scratch need above the maximum. */
+ * Errors: as lq_gemm, plus LQ_EINVAL for batch > 8 or a scratch need above the maximum, and
+ * LQ_EUNSUPPORTED when no single-launch GEMV plan fits the shape (its K-slices cannot widen
+ * enough for a CTA's rows to fit its warps' partial slots, e.g. 5..8 tokens of a 28672-row
+ * layer); lq_gemm runs such batches as token groups. */
 LQ_API lq_status lq_gemm_noalloc(const void* x, lq_dtype xdt, int32_t batch,
                                  const lq_whiten_desc* T, const uint32_t* packed, const float* M,
                                  const void* s, lq_dtype sdt, int32_t d, int32_t D, int32_t K,
