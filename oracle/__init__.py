@@ -51,6 +51,8 @@ def _load(path=None):
     lib.orc_encode_rows.restype = ctypes.c_int
     lib.orc_codebook_round.argtypes = [_dp, i64, _dp, i32, i32, i32, _i8p, ctypes.c_int]
     lib.orc_codebook_round.restype = ctypes.c_double
+    lib.orc_codebook_refit.argtypes = [_dp, i64, _i8p, _dp, i32, i32]
+    lib.orc_codebook_refit.restype = ctypes.c_int
     lib.orc_max_threads.argtypes = []
     lib.orc_max_threads.restype = ctypes.c_int
     return lib
@@ -249,6 +251,19 @@ def codebook_round(w, M, d, D, mode=0, nthreads=0, _lib=None):
     if mse < 0:
         raise ValueError("oracle codebook_round rejected its arguments")
     return Mf, b, float(mse)
+
+
+def codebook_refit(w, b, M, d, D, _lib=None):
+    """The least-squares step of the codebook fit alone: M = (sum w b^T)(sum b b^T)^-1 for the
+    samples w [S][d] and their codes b [S][D] (+-1). Returns M_new [d][D] (M gives its shape
+    and is not modified)."""
+    L = _lib or lib()
+    wf = _f64(w).reshape(-1, d)
+    bb = np.ascontiguousarray(b, dtype=np.int8).reshape(wf.shape[0], D)
+    Mf = _f64(M).reshape(d, D).copy()
+    if L.orc_codebook_refit(_ptr(wf, _dp), wf.shape[0], _ptr(bb, _i8p), _ptr(Mf, _dp), d, D) != 0:
+        raise ValueError("oracle codebook_refit rejected its arguments (or sum b b^T is singular)")
+    return Mf
 
 
 def max_threads(_lib=None):

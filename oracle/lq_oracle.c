@@ -431,27 +431,87 @@ int orc_encode_rows(const double* w, int64_t N, int32_t K, const double* M, int3
   return failed ? -1 : 0;
 }
 
+/* The least-squares step of the codebook fit (review "Method": M is fitted offline to a
+ * standard Gaussian; paper sec. 3.1, Eq. (1)): with the codes b_s of the samples w_s [S][d]
+ * fixed, M [d][D] becomes M = (sum_s w_s b_s^T)(sum_s b_s b_s^T)^-1, the point where the
+ * straight-through gradient -2 sum_s (w_s - M b_s) b_s^T vanishes. Sums run in sample order in
+ * fp64; the D x D system is solved by elimination with partial pivoting. Returns 0, or -1 for
+ * invalid sizes or a singular sum b b^T (M is then left unchanged). */
+int orc_codebook_refit(const double* w, int64_t S, const int8_t* b, double* M, int32_t d,
+                       int32_t D) {
+  if (S < 1 || d < 1 || D < d || D > 32) return -1;
+  double* A = (double*)calloc((size_t)d * (size_t)D, sizeof(double));
+  double* C = (double*)calloc((size_t)D * (size_t)(D + d), sizeof(double));
+  if (!A || !C) {
+    free(A);
+    free(C);
+    return -1;
+  }
+  int rc = 0;
+  /* sums in sample order: A = sum w b^T [d][D]; the system C^T X = A^T with C = sum b b^T,
+   * stored augmented as [D][D + d] */
+  for (int64_t n = 0; n < S; ++n) {
+    const int8_t* bn = b + n * D;
+    for (int32_t i = 0; i < d; ++i)
+      for (int32_t j = 0; j < D; ++j) A[i * D + j] += w[n * d + i] * (double)bn[j];
+    for (int32_t j = 0; j < D; ++j)
+      for (int32_t k = 0; k < D; ++k) C[j * (D + d) + k] += (double)bn[j] * (double)bn[k];
+  }
+  for (int32_t j = 0; j < D; ++j)
+    for (int32_t i = 0; i < d; ++i) C[j * (D + d) + D + i] = A[i * D + j];
+  /* C is symmetric: solve C X = A^T (X = M^T) by elimination with partial pivoting */
+  const int32_t W = D + d;
+  for (int32_t c = 0; c < D && rc == 0; ++c) {
+    int32_t piv = c;
+    for (int32_t r = c + 1; r < D; ++r)
+      if (fabs(C[r * W + c]) > fabs(C[piv * W + c])) piv = r;
+    if (fabs(C[piv * W + c]) < 1e-12 * (double)S) {
+      rc = -1;
+      break;
+    }
+    if (piv != c)
+      for (int32_t k = 0; k < W; ++k) {
+        const double t = C[c * W + k];
+        C[c * W + k] = C[piv * W + k];
+        C[piv * W + k] = t;
+      }
+    for (int32_t r = c + 1; r < D; ++r) {
+      const double m = C[r * W + c] / C[c * W + c];
+      for (int32_t k = c; k < W; ++k) C[r * W + k] -= m * C[c * W + k];
+    }
+  }
+  if (rc == 0) {
+    for (int32_t i = 0; i < d; ++i)
+      for (int32_t c = D - 1; c >= 0; --c) {
+        double x = C[c * W + D + i];
+        for (int32_t k = c + 1; k < D; ++k) x -= C[c * W + k] * C[k * W + D + i];
+        x /= C[c * W + c];
+        C[c * W + D + i] = x;            /* X[c][i] = M[i][c] */
+      }
+    for (int32_t i = 0; i < d; ++i)
+      for (int32_t c = 0; c < D; ++c) M[i * D + c] = C[c * W + D + i];
+  }
+  free(A);
+  free(C);
+  return rc;
+}
+
 /* One round of the codebook optimisation: M is fitted offline to a standard Gaussian (review
  * "Method"; paper sec. 3.1, Eq. (1), whose text is cut before the gradient path through the
  * encoder). Reading: alternating minimisation of the mean of ||w - M b(w)||^2 over samples
  * w_s [S][d]: (1) every sample takes its nearest codeword under the current M (mode 0
  * exhaustive, 1 seeded); (2) with the codes fixed, M becomes the least-squares fit
- * M = (sum_s w_s b_s^T)(sum_s b_s b_s^T)^-1, the point where the straight-through gradient
- * -2 sum_s (w_s - M b_s) b_s^T vanishes. M [d][D] is updated in place; b_out [S][D] (optional)
- * receives the codes of step (1). Returns the mean squared error per weight of step (1), or -1
- * for invalid input or a singular sum b b^T (M is then left unchanged). */
+ * (orc_codebook_refit). M [d][D] is updated in place; b_out [S][D] (optional) receives the
+ * codes of step (1). Returns the mean squared error per weight of step (1), or -1 for invalid
+ * input or a singular sum b b^T (M is then left unchanged). */
 double orc_codebook_round(const double* w, int64_t S, double* M, int32_t d, int32_t D,
                           int32_t mode, int8_t* b_out, int nthreads) {
   if (S < 1 || d < 1 || D < d || D > 24 || (mode != 0 && mode != 1)) return -1.0;
   int8_t* b = b_out ? b_out : (int8_t*)malloc((size_t)S * (size_t)D);
   double* err = (double*)malloc(sizeof(double) * (size_t)S);
-  double* A = (double*)calloc((size_t)d * (size_t)D, sizeof(double));
-  double* C = (double*)calloc((size_t)D * (size_t)(D + d), sizeof(double));
-  if (!b || !err || !A || !C) {
+  if (!b || !err) {
     if (!b_out) free(b);
     free(err);
-    free(A);
-    free(C);
     return -1.0;
   }
   int failed = 0;
@@ -472,54 +532,10 @@ double orc_codebook_round(const double* w, int64_t S, double* M, int32_t d, int3
     double tot = 0.0;
     for (int64_t n = 0; n < S; ++n) tot += err[n];
     mse = tot / ((double)S * d);
-    /* sums in sample order: A = sum w b^T [d][D]; the system C^T X = A^T with C = sum b b^T,
-     * stored augmented as [D][D + d] */
-    for (int64_t n = 0; n < S; ++n) {
-      const int8_t* bn = b + n * D;
-      for (int32_t i = 0; i < d; ++i)
-        for (int32_t j = 0; j < D; ++j) A[i * D + j] += w[n * d + i] * (double)bn[j];
-      for (int32_t j = 0; j < D; ++j)
-        for (int32_t k = 0; k < D; ++k) C[j * (D + d) + k] += (double)bn[j] * (double)bn[k];
-    }
-    for (int32_t j = 0; j < D; ++j)
-      for (int32_t i = 0; i < d; ++i) C[j * (D + d) + D + i] = A[i * D + j];
-    /* C is symmetric: solve C X = A^T (X = M^T) by elimination with partial pivoting */
-    const int32_t W = D + d;
-    for (int32_t c = 0; c < D && mse >= 0.0; ++c) {
-      int32_t piv = c;
-      for (int32_t r = c + 1; r < D; ++r)
-        if (fabs(C[r * W + c]) > fabs(C[piv * W + c])) piv = r;
-      if (fabs(C[piv * W + c]) < 1e-12 * (double)S) {
-        mse = -1.0;
-        break;
-      }
-      if (piv != c)
-        for (int32_t k = 0; k < W; ++k) {
-          const double t = C[c * W + k];
-          C[c * W + k] = C[piv * W + k];
-          C[piv * W + k] = t;
-        }
-      for (int32_t r = c + 1; r < D; ++r) {
-        const double m = C[r * W + c] / C[c * W + c];
-        for (int32_t k = c; k < W; ++k) C[r * W + k] -= m * C[c * W + k];
-      }
-    }
-    if (mse >= 0.0) {
-      for (int32_t i = 0; i < d; ++i)
-        for (int32_t c = D - 1; c >= 0; --c) {
-          double x = C[c * W + D + i];
-          for (int32_t k = c + 1; k < D; ++k) x -= C[c * W + k] * C[k * W + D + i];
-          x /= C[c * W + c];
-          C[c * W + D + i] = x;            /* X[c][i] = M[i][c] */
-        }
-      for (int32_t i = 0; i < d; ++i)
-        for (int32_t c = 0; c < D; ++c) M[i * D + c] = C[c * W + D + i];
-    }
+    if (orc_codebook_refit(w, S, b, M, d, D) != 0) mse = -1.0;
   }
   if (!b_out) free(b);
   free(err);
-  free(A);
-  free(C);
   return mse;
 }
 

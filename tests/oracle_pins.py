@@ -461,4 +461,27 @@ def pin_codebook_round(orc):
         last = m
 
 
+def pin_codebook_refit(orc):
+    """The least-squares step alone, against numpy's least-squares solver of min ||W - B M^T||
+    (not the normal equations the oracle forms), on random codes up to D = 32; with the codes of
+    a round it reproduces that round's M; a codebook whose sum b b^T is singular is rejected."""
+    rng = _rng(23)
+    for d, D, S in [(1, 2, 50), (2, 5, 400), (10, 24, 3000), (16, 32, 5000)]:
+        w = rng.standard_normal((S, d))
+        b = np.where(rng.random((S, D)) < 0.5, -1, 1).astype(np.int8)
+        M = orc.codebook_refit(w, b, np.zeros((d, D)), d, D)
+        ref = np.linalg.lstsq(b.astype(np.float64), w, rcond=None)[0].T
+        assert np.allclose(M, ref, atol=1e-10, rtol=1e-9), (d, D)
+    w = rng.standard_normal((300, 2))
+    M0 = rng.standard_normal((2, 5)) * 0.5
+    M1, b, _ = orc.codebook_round(w, M0, 2, 5)
+    assert np.allclose(orc.codebook_refit(w, b, M0, 2, 5), M1, atol=1e-13)
+    same = np.ones((40, 3), dtype=np.int8)          # every code equal: sum b b^T has rank 1
+    try:
+        orc.codebook_refit(rng.standard_normal((40, 2)), same, np.zeros((2, 3)), 2, 3)
+        raise AssertionError("a singular sum b b^T was accepted")
+    except ValueError:
+        pass
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
