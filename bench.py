@@ -1,10 +1,12 @@
 """Benchmark of the LiftQuant decode operator (lq_gemm) on B200.
 
 One step = one lq_gemm call (whiten + lift + +-1 contraction + row scale) over one batch of
-synthetic inputs already resident in HBM. The default workload is the Llama-2-7B q_proj
-shape (K = N = 4096, d = 10, D = 24: 2.4 bit, batch 1, block-256 Hadamard whitening).
-Inputs rotate over enough copies of the packed weights that successive steps never hit in
-L2. Prints one JSON line (rank 0).
+synthetic inputs already resident in HBM. The default workload is the Llama-3-70B MLP
+gate/up shape (K = 8192 -> N = 28672, d = 10, D = 24: 2.4 bit, batch 1, block-256 Hadamard
+whitening), the batch-1 GEMV whose packed-weight bandwidth is the headline; the same run then
+times the 2048-token prefill GEMM of that layer (TFLOP/s, nested as "prefill"). Inputs rotate
+over enough copies of the packed weights that no timed step finds its codes in L2. Prints one
+JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl lq|reference]
 
@@ -47,6 +49,11 @@ WORKLOADS = {
     # encoder: 512 rows of the q_proj shape, seeded 2^(D-d) search per block
     "encode_seeded_512x4096_d10D24": (None, None, "encode"),
 }
+PREFILL = "prefill_b2048"
+# --route: lq_gemm's own choice, or one kernel family through lq_gemm_on_route
+ROUTES = {"auto": None, "gemv_i8": lq.ROUTE_GEMV_I8, "gemm_tc": lq.ROUTE_GEMM_TC,
+          "gemv_groups": lq.ROUTE_GEMV_GROUPS, "gemv_bulk": lq.ROUTE_GEMV_BULK,
+          "gemm_dq": lq.ROUTE_GEMM_DQ}
 
 # the encoder workload: (N, K, d, D, mode, seed); w ~ N(0, 1) stands for whitened weights,
 # M ~ N(0, 1/D)
@@ -61,7 +68,12 @@ def parse():
     p.add_argument("--steps", type=int, default=2000)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", default="lq", choices=["lq", "reference"])
-    p.add_argument("--workload", default="llama2_7b_qproj_b1", choices=sorted(WORKLOADS))
+    p.add_argument("--workload", default="llama3_70b_gateup_b1", choices=sorted(WORKLOADS))
+    p.add_argument("--prefill-steps", type=int, default=10,
+                   help="steps of the 2048-token prefill GEMM timed after a GEMV workload "
+                        "(reported as the nested 'prefill' object; 0 skips it)")
+    p.add_argument("--route", default="auto", choices=sorted(ROUTES),
+                   help="kernel family for the lq_gemm call (auto: the library's choice)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     return p.parse_args()
@@ -108,9 +120,10 @@ def source_digest(name):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def recorded_traffic(workload):
-    """DRAM bytes per launch of the workload's dominant kernel from profiles/traffic.json (an
-    ncu capture), if the file defining that kernel is unchanged since (else None)."""
+def recorded_traffic(workload, field):
+    """A figure of the workload's dominant kernel from profiles/traffic.json (an ncu capture:
+    DRAM bytes per launch, tensor-pipe activity), if the file defining that kernel is
+    unchanged since (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -123,7 +136,7 @@ def recorded_traffic(workload):
             return None
     except (OSError, KeyError):
         return None
-    return ent.get("dram_bytes_per_launch")
+    return ent.get(field)
 
 
 class ClockSampler:
@@ -190,7 +203,7 @@ class ClockSampler:
 # ---------------------------------------------------------------- workload on the device
 
 class DeviceWorkload:
-    def __init__(self, spec, dev):
+    def __init__(self, spec, dev, min_copies=1, route=None):
         name, seed, li, K, N, d, D, batch, kw = spec
         self.name, self.K, self.N, self.d, self.D, self.batch = name, K, N, d, D, batch
         layer = synth.build(spec, with_bits=False)     # sign, M, s, x from the seeded recipe
@@ -203,7 +216,7 @@ class DeviceWorkload:
         g.manual_seed(seed * 1000 + li)
         # rotate over copies so that the bytes streamed between reuses exceed 3x L2
         stored = N * self.row_words * 4
-        self.ncopies = max(1, min(64, math.ceil(3 * L2_BYTES / stored)))
+        self.ncopies = max(min_copies, min(64, math.ceil(3 * L2_BYTES / stored)))
         self.packed = []
         for _ in range(self.ncopies):
             b = (torch.randint(0, 2, (N, self.L), generator=g, device=dev, dtype=torch.int8)
@@ -215,13 +228,14 @@ class DeviceWorkload:
         self.M = torch.from_numpy(layer.M).to(dev)
         self.sign = torch.from_numpy(layer.sign).to(dev)
         self.y = torch.empty((batch, N), dtype=torch.float32, device=dev)
-        self.ws = lq.new_workspace(batch, K, N, d, D, device=dev)
+        self.route = route
+        self.ws = lq.new_workspace(batch, K, N, d, D, device=dev, block=self.block, route=route)
         self.stored_bytes = stored
 
     def step(self, i, x=None, y=None):
         lq.gemm(self.x if x is None else x, self.packed[i % self.ncopies], self.M, self.s,
                 self.d, self.D, sign=self.sign, block=self.block,
-                y=self.y if y is None else y, workspace=self.ws)
+                y=self.y if y is None else y, workspace=self.ws, route=self.route)
 
     def algorithmic_bytes(self):
         """Bytes one call must move at minimum: packed codes, s, x, y, M, sign."""
@@ -230,10 +244,27 @@ class DeviceWorkload:
                 + self.M.numel() * 4 + self.sign.numel())
 
     def flops(self):
-        """Contraction + lift + FWHT flops of one call (lifted form)."""
+        """The method's algorithmic flops of one call: the lifted contraction (2 B N L) plus the
+        lift and the FWHT."""
         G = -(-self.K // self.d)
         fwht = self.batch * self.K * int(math.log2(self.block)) if self.block else 0
         return 2.0 * self.batch * self.N * self.L + 2.0 * self.batch * G * self.d * self.D + fwht
+
+    def actual_route(self):
+        if self.route is not None:
+            return self.route
+        return lq.gemm_route(self.batch, self.K, self.N, self.d, self.D, self.block)
+
+    def tensor_flops(self):
+        """Tensor-core flops the route's contraction kernel executes per call: the lifted GEMM
+        2 B N Lp (L padded to its 64-coordinate stage); the dequantise-once GEMM 2 B N Kw (the
+        G*d inputs padded to 64), which is D/d times fewer than the lifted count."""
+        if self.actual_route() == lq.ROUTE_GEMM_DQ:
+            G = -(-self.K // self.d)
+            Kw = -(-(G * self.d) // 64) * 64
+            return 2.0 * self.batch * self.N * Kw
+        Lp = -(-self.L // 64) * 64
+        return 2.0 * self.batch * self.N * Lp
 
 
 def _x_tensor(layer):
@@ -243,42 +274,60 @@ def _x_tensor(layer):
 
 
 def kernels_per_step(wl):
-    """Kernels one lq_gemm call launches for this workload, as the library reports it."""
+    """Kernels one lq_gemm call launches for this workload: as the library reports it, or on a
+    forced route its fixed count (bulk GEMV 1; int8 GEMV and lifted GEMM 2; W, xt, GEMM 3)."""
+    fixed = {lq.ROUTE_GEMV_BULK: 1, lq.ROUTE_GEMV_I8: 2, lq.ROUTE_GEMM_TC: 2, lq.ROUTE_GEMM_DQ: 3}
+    if wl.route in fixed:
+        return fixed[wl.route]
     return lq.gemm_launches(wl.batch, wl.K, wl.N, wl.d, wl.D, wl.block)
 
 
-def time_steps(fn, steps, warmup, ws, graph_block=None):
+def time_steps(fn, steps, warmup, ws, ncopies=None):
     """Device time of exactly `steps` calls of fn(i), after `warmup` untimed calls.
 
-    With graph_block, the calls are captured into CUDA graphs of graph_block steps (plus one
-    graph for the remainder) and replayed, so host launch overhead stays out of the timing."""
+    With ncopies (the number of rotating input copies, fn(i) reading copy i % ncopies), the
+    calls are captured into CUDA graphs and replayed, so host launch overhead stays out of the
+    timing: one graph over all copies in order (0 .. ncopies-1) and, when steps is not a
+    multiple of ncopies, one over copies 0 .. (steps % ncopies)-1. The warm replay ends with
+    the full graph, so the first timed step reads copy 0, which was last read ncopies - 1 steps
+    earlier; every timed step reads a copy that ncopies - 1 other copies were streamed after.
+    Returns (seconds, the smallest number of other copies read between two reads of a copy)."""
     for i in range(warmup):
         fn(i)
     torch.cuda.synchronize()
-    graphs = []
-    if graph_block:
-        gb = max(1, min(graph_block, steps))
-        sizes = [gb] * (steps // gb) + ([steps % gb] if steps % gb else [])
-        cache = {}
-        base = warmup
-        for n in sizes:
-            if n not in cache:
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g):
-                    for i in range(n):
-                        fn(base + i)
-                cache[n] = g
-            graphs.append(cache[n])
-        for g in cache.values():          # warm the graphs
-            g.replay()
+    plan = []
+    reuse = None
+    if ncopies:
+        full, rem = divmod(steps, ncopies)
+        g_full = g_rem = None
+        if full:
+            g_full = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_full):
+                for i in range(ncopies):
+                    fn(i)
+        if rem:
+            g_rem = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_rem):
+                for i in range(rem):
+                    fn(i)
+        if g_rem is not None:
+            g_rem.replay()
+        # the warm-up ends with a pass over every copy in order (eager if no full graph)
+        if g_full is not None:
+            g_full.replay()
+        else:
+            for i in range(ncopies):
+                fn(i)
         torch.cuda.synchronize()
+        plan = [g_full] * full + ([g_rem] if g_rem is not None else [])
+        reuse = ncopies - 1
     barrier(ws)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    if graphs:
-        for g in graphs:
+    if plan:
+        for g in plan:
             g.replay()
     else:
         for i in range(steps):
@@ -287,8 +336,8 @@ def time_steps(fn, steps, warmup, ws, graph_block=None):
     torch.cuda.synchronize()
     barrier(ws)
     torch.cuda.synchronize()
-    del graphs
-    return e0.elapsed_time(e1) / 1e3   # seconds
+    del plan
+    return e0.elapsed_time(e1) / 1e3, reuse   # seconds
 
 
 # ---------------------------------------------------------------- CPU oracle baseline
@@ -325,6 +374,61 @@ def cpu_oracle_run(wl, budget_s=10.0, max_rows=None):
 
 # ---------------------------------------------------------------- main
 
+def measure(wl, name, kind, steps, warmup, ws, local, peaks, peak_src):
+    """Times `steps` calls of the workload (inputs resident in HBM) and returns the headline
+    fields of its JSON line."""
+    with ClockSampler(local) as clk:
+        secs, reuse = time_steps(wl.step, steps, warmup, ws, ncopies=wl.ncopies)
+    secs = max_over_ranks(secs, ws)
+    per_step = secs / steps
+    gbs = wl.packed_bytes * steps * ws / secs / 1e9
+    tflops = wl.flops() * steps * ws / secs / 1e12
+    if kind == "gemv":
+        metric, value, unit = "lq_gemv_packed_weight_GBps", gbs, "GB/s"
+        achieved = wl.algorithmic_bytes() / per_step / 1e9
+        peak = float(peaks["hbm_gbs"])
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": recorded_traffic(name, "dram_bytes_per_launch"),
+                "peak_source": f"{peak_src} hbm_gbs (copy, read+write)",
+                "packed_frac": wl.packed_bytes / per_step / 1e9 / peak}
+    else:
+        # value: the method's algorithmic (lifted) flops per second, comparable across routes;
+        # roofline: the flops the tensor cores actually execute on this route, per second of
+        # the whole call (all its kernels), against the measured dense peak
+        metric, value, unit = "lq_prefill_gemm_TFLOPs", tflops, "TFLOP/s"
+        achieved = wl.tensor_flops() / per_step / 1e12
+        # the burst figure: the timed region is short and the clocks stay at their maximum
+        # (the sampled clocks are in the same line); fp16 dense rate = bf16 dense rate
+        peak = float(peaks.get("bf16_tflops", peaks.get("bf16_tflops_sustained")))
+        route = wl.actual_route()
+        rname = {lq.ROUTE_GEMM_TC: "lifted tcgen05 GEMM", lq.ROUTE_GEMM_DQ:
+                 "dequantise-once: fp16 W = M b, then a dense tcgen05 GEMM"}.get(route, str(route))
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": recorded_traffic(name, "dram_bytes_per_launch"),
+                "tensor_pipe_active": recorded_traffic(name, "tensor_pipe_active"),
+                "route": rname, "executed_tensor_flops": wl.tensor_flops(),
+                "algorithmic_flops": wl.flops(),
+                "peak_source": f"{peak_src} bf16_tflops (burst; fp16 dense = bf16 dense)"}
+    streamed = reuse * wl.stored_bytes
+    l2 = (f"{wl.ncopies} copies of the packed weights ({wl.ncopies * wl.stored_bytes / 1e6:.0f} "
+          f"MB) read in rotation, warm-up included: between two reads of a copy "
+          f"{reuse} other copies ({streamed / 1e6:.0f} MB"
+          f"{' > L2' if streamed > L2_BYTES else ' <= L2'}) are streamed")
+    if kind == "gemm":
+        l2 += f"; y alone is {wl.y.numel() * 4 / 1e6:.0f} MB per step"
+    return {
+        "metric": metric, "value": value, "unit": unit, "ms_per_step": per_step * 1e3,
+        "config": {"workload": wl.name, "K": wl.K, "N": wl.N, "d": wl.d, "D": wl.D,
+                   "batch": wl.batch, "bits_per_weight": wl.D / wl.d, "hadamard_block": wl.block,
+                   "packed_bytes": wl.packed_bytes, "parallelism": f"replicas x{ws}",
+                   "l2": l2},
+        "roofline": roof,
+        "gpu_launches": kernels_per_step(wl) * steps,
+        "clocks": clk.summary(),
+        "tflops": tflops,
+    }
+
+
 def main():
     args = parse()
     ws, rank, local = dist_setup()
@@ -337,60 +441,44 @@ def main():
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    wl = DeviceWorkload(spec, dev)
+    wl = DeviceWorkload(spec, dev, route=ROUTES[args.route])
     peaks, peak_src = measured_peaks()
-
-    with ClockSampler(local) as clk:
-        secs = time_steps(wl.step, args.steps, args.warmup, ws, graph_block=wl.ncopies)
-    secs = max_over_ranks(secs, ws)
-    per_step = secs / args.steps
-
-    total_packed = wl.packed_bytes * args.steps * ws
-    gbs = total_packed / secs / 1e9
-    tflops = wl.flops() * args.steps * ws / secs / 1e12
-    if kind == "gemv":
-        metric, value, unit = "lq_gemv_packed_weight_GBps", gbs, "GB/s"
-        achieved = wl.algorithmic_bytes() / per_step / 1e9
-        peak = float(peaks["hbm_gbs"])
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
-                "peak_source": f"{peak_src} hbm_gbs (copy, read+write)",
-                "packed_frac": wl.packed_bytes / per_step / 1e9 / peak}
-    else:
-        metric, value, unit = "lq_prefill_gemm_TFLOPs", tflops, "TFLOP/s"
-        achieved = wl.flops() / per_step / 1e12
-        # the burst figure: the timed region is short and the clocks stay at their maximum
-        # (the sampled clocks are in the same line); fp16 dense rate = bf16 dense rate
-        peak = float(peaks.get("bf16_tflops", peaks.get("bf16_tflops_sustained")))
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
-                "peak_source": f"{peak_src} bf16_tflops (burst; fp16 dense = bf16 dense)"}
+    m = measure(wl, args.workload, kind, args.steps, args.warmup, ws, local, peaks, peak_src)
 
     out = {
-        "metric": metric, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "metric": m["metric"], "value": m["value"], "unit": m["unit"], "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": m["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded: random sign codes, N(0,1/D) M, N(0,1) bf16 x)",
-        "config": {"workload": wl.name, "K": wl.K, "N": wl.N, "d": wl.d, "D": wl.D,
-                   "batch": wl.batch, "bits_per_weight": wl.D / wl.d, "hadamard_block": wl.block,
-                   "packed_bytes": wl.packed_bytes, "parallelism": f"replicas x{ws}",
-                   "l2": f"rotating {wl.ncopies} copies of the packed weights "
-                         f"({wl.ncopies * wl.stored_bytes / 1e6:.0f} MB > L2)"},
-        "roofline": roof,
-        "gpu_launches": kernels_per_step(wl) * args.steps,
+        "config": m["config"],
+        "roofline": m["roofline"],
+        "gpu_launches": m["gpu_launches"],
         "timing": "CUDA graphs of the steps, replayed; CUDA events on the launching stream",
-        "clocks": clk.summary(),
+        "clocks": m["clocks"],
     }
     if kind == "gemv":
-        out["tflops"] = tflops
+        out["tflops"] = m["tflops"]
     if not args.no_e2e:
         out["e2e"] = e2e_run(wl, args, ws)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         frac, dt, sample, threads = cpu_oracle_run(wl)
         cpu_val = (wl.packed_bytes * frac / dt / 1e9) if kind == "gemv" else \
             (wl.flops() * frac / dt / 1e12)
-        out["cpu_baseline"] = {"value": cpu_val, "unit": unit, "cores": threads, "kind": "oracle",
-                               "sample": sample}
+        out["cpu_baseline"] = {"value": cpu_val, "unit": m["unit"], "cores": threads,
+                               "kind": "oracle", "sample": sample}
+    del wl
+    if args.prefill_steps > 0 and kind == "gemv":
+        # the second half of the metric: the 2048-token prefill GEMM, timed in the same run
+        pcfg, pidx, _ = WORKLOADS[PREFILL]
+        pwl = DeviceWorkload(synth.workload_specs(pcfg)[pidx], dev, min_copies=2)
+        p = measure(pwl, PREFILL, "gemm", args.prefill_steps, max(3, args.warmup // 4), ws,
+                    local, peaks, peak_src)
+        out["prefill"] = {"metric": p["metric"], "value": p["value"], "unit": p["unit"],
+                          "steps": args.prefill_steps, "ms_per_step": p["ms_per_step"],
+                          "config": p["config"], "roofline": p["roofline"],
+                          "gpu_launches": p["gpu_launches"], "clocks": p["clocks"]}
+        out["gpu_launches"] += p["gpu_launches"]
+        del pwl
     if rank == 0:
         print(json.dumps(out))
     if ws > 1:
@@ -460,7 +548,7 @@ def encode_main(args, ws, rank, local):
             raise RuntimeError(lib.lq_last_error().decode())
 
     with ClockSampler(local) as clk:
-        secs = time_steps(step, args.steps, args.warmup, ws)
+        secs, _ = time_steps(step, args.steps, args.warmup, ws)
     secs = max_over_ranks(secs, ws)
     per_step = secs / args.steps
     value = N * K * args.steps * ws / secs
@@ -492,7 +580,7 @@ def encode_main(args, ws, rank, local):
             step(i, w_dev)
             b_host.copy_(b, non_blocking=True)
 
-        e2e_secs = max_over_ranks(time_steps(e2e_step, args.steps, args.warmup, ws), ws)
+        e2e_secs = max_over_ranks(time_steps(e2e_step, args.steps, args.warmup, ws)[0], ws)
         out["e2e"] = {"value": N * K * args.steps * ws / e2e_secs, "unit": "weights/s",
                       "h2d_bytes_per_step": N * K * 4, "d2h_bytes_per_step": N * G * D}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -517,7 +605,7 @@ def e2e_run(wl, args, ws):
         wl.step(i, x=x_dev)
         y_host.copy_(wl.y, non_blocking=True)
 
-    secs = max_over_ranks(time_steps(step, args.steps, args.warmup, ws), ws)
+    secs = max_over_ranks(time_steps(step, args.steps, args.warmup, ws)[0], ws)
     if wl.flops() and WORKLOADS[args.workload][2] == "gemm":
         v, u = wl.flops() * args.steps * ws / secs / 1e12, "TFLOP/s"
     else:

@@ -28,7 +28,9 @@ LQ_F32, LQ_F16, LQ_BF16 = 0, 1, 2
 _DTYPES = {torch.float32: LQ_F32, torch.float16: LQ_F16, torch.bfloat16: LQ_BF16}
 
 EXPORTS = ("lq_abi_version", "lq_lifted_bits", "lq_row_stride_bytes", "lq_pack", "lq_unpack", "lq_encode",
-           "lq_whiten", "lq_lift", "lq_gemm_workspace_bytes", "lq_gemm_launches", "lq_gemm",
+           "lq_whiten", "lq_lift", "lq_gemm_workspace_bytes", "lq_gemm_launches", "lq_gemm_route",
+           "lq_gemm", "lq_gemm_on_route", "lq_gemm_route_workspace_bytes",
+           "lq_codebook_workspace_bytes", "lq_codebook_round",
            "lq_gemm_noalloc", "lq_check_wait_timeout",
            "lq_device_status", "lq_status_string", "lq_last_error")
 
@@ -61,8 +63,15 @@ def _declare(L):
         "lq_lift": ([vp, ctypes.c_int, i32, i32, dp, vp, i32, i32, vp, vp], ctypes.c_int),
         "lq_gemm_workspace_bytes": ([i32, i32, i32, i32, i32], sz),
         "lq_gemm_launches": ([i32, i32, i32, i32, i32, i32], i32),
+        "lq_gemm_route": ([i32, i32, i32, i32, i32, i32], i32),
         "lq_gemm": ([vp, ctypes.c_int, i32, dp, vp, vp, vp, ctypes.c_int, i32, i32, i32, i32, vp,
                      vp, sz, vp], ctypes.c_int),
+        "lq_gemm_on_route": ([vp, ctypes.c_int, i32, dp, vp, vp, vp, ctypes.c_int, i32, i32, i32,
+                              i32, vp, vp, sz, i32, vp], ctypes.c_int),
+        "lq_gemm_route_workspace_bytes": ([i32, i32, i32, i32, i32, i32, i32], sz),
+        "lq_codebook_workspace_bytes": ([ctypes.c_int64, i32, i32], sz),
+        "lq_codebook_round": ([vp, ctypes.c_int64, vp, i32, i32, i32, vp, vp, vp, sz, vp],
+                              ctypes.c_int),
         "lq_gemm_noalloc": ([vp, ctypes.c_int, i32, dp, vp, vp, vp, ctypes.c_int, i32, i32, i32,
                              i32, vp, vp], ctypes.c_int),
         "lq_device_status": ([vp, ctypes.POINTER(i32), vp], ctypes.c_int),
@@ -205,30 +214,50 @@ def gemm_launches(batch, K, N, d, D, block=0):
     return int(lib().lq_gemm_launches(batch, K, N, d, D, block))
 
 
-def new_workspace(batch, K, N, d, D, device="cuda"):
-    """A zero-filled workspace tensor for lq_gemm (uint8, 256-byte aligned by torch)."""
-    n = gemm_workspace_bytes(batch, K, N, d, D)
+# lq_gemm_route codes (include/liblq.h)
+ROUTE_GEMV_I8, ROUTE_NONE, ROUTE_GEMM_TC, ROUTE_GEMV_GROUPS, ROUTE_GEMV_BULK, ROUTE_GEMM_DQ = \
+    0, 1, 2, 3, 4, 5
+
+
+def gemm_route(batch, K, N, d, D, block=0):
+    """Which kernels lq_gemm runs for this shape (host-only query; ROUTE_* codes)."""
+    return int(lib().lq_gemm_route(batch, K, N, d, D, block))
+
+
+def new_workspace(batch, K, N, d, D, device="cuda", block=0, route=None):
+    """A zero-filled workspace tensor for lq_gemm (uint8, 256-byte aligned by torch); with a
+    route, for lq_gemm_on_route on that route and Hadamard block."""
+    if route is None:
+        n = gemm_workspace_bytes(batch, K, N, d, D)
+    else:
+        n = int(lib().lq_gemm_route_workspace_bytes(batch, K, N, d, D, block, int(route)))
     if n == 0:
         raise ValueError("invalid sizes for lq_gemm")
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def gemm(x, packed, M, s, d, D, sign=None, chan_scale=None, block=0, y=None, workspace=None,
-         stream=None):
-    """y[t][n] = s[n] * (W[n] . T(x[t])), float32 [batch][N]."""
+         stream=None, route=None):
+    """y[t][n] = s[n] * (W[n] . T(x[t])), float32 [batch][N].
+
+    route=None lets the library pick the kernels (lq_gemm); a ROUTE_* code runs that route
+    (lq_gemm_on_route), which must fit the shape."""
     batch, K = x.shape
     N = packed.shape[0]
     if y is None:
         y = torch.empty((batch, N), dtype=torch.float32, device=x.device)
     if workspace is None:
-        workspace = new_workspace(batch, K, N, d, D, device=x.device)
+        workspace = new_workspace(batch, K, N, d, D, device=x.device, block=block, route=route)
     desc = _whiten_desc(sign, chan_scale, block)
-    _check(lib().lq_gemm(_dev(x, "x", _DTYPES), _DTYPES[x.dtype], batch, _desc_ptr(desc),
-                         _dev(packed, "packed", (torch.int32,)), _dev(M, "M", (torch.float32,)),
-                         _dev(s, "s", _DTYPES), _DTYPES[s.dtype], d, D, K, N,
-                         _dev(y, "y", (torch.float32,)), _dev(workspace, "workspace"),
-                         workspace.numel() * workspace.element_size(), _stream(stream)),
-           "lq_gemm")
+    args = (_dev(x, "x", _DTYPES), _DTYPES[x.dtype], batch, _desc_ptr(desc),
+            _dev(packed, "packed", (torch.int32,)), _dev(M, "M", (torch.float32,)),
+            _dev(s, "s", _DTYPES), _DTYPES[s.dtype], d, D, K, N,
+            _dev(y, "y", (torch.float32,)), _dev(workspace, "workspace"),
+            workspace.numel() * workspace.element_size())
+    if route is None:
+        _check(lib().lq_gemm(*args, _stream(stream)), "lq_gemm")
+    else:
+        _check(lib().lq_gemm_on_route(*args, int(route), _stream(stream)), "lq_gemm_on_route")
     return y
 
 
@@ -251,6 +280,29 @@ def gemm_noalloc(x, packed, M, s, d, D, sign=None, chan_scale=None, block=0, y=N
                                  _DTYPES[s.dtype], d, D, K, N, _dev(y, "y", (torch.float32,)),
                                  _stream(stream)), "lq_gemm_noalloc")
     return y
+
+
+def codebook_round(w, M, d, D, mode=0, b=None, mse=None, workspace=None, stream=None):
+    """One round of the codebook fit on samples w [S][d] (fp32, device): nearest codewords
+    under M, then the least-squares M. M (fp32 [d][D], device) is updated in place. Returns
+    (M, codes int8 [S][D], mse fp64 tensor of one element) on the device."""
+    S = w.shape[0]
+    if b is None:
+        b = torch.empty((S, D), dtype=torch.int8, device=w.device)
+    if mse is None:
+        mse = torch.empty(1, dtype=torch.float64, device=w.device)
+    if workspace is None:
+        n = int(lib().lq_codebook_workspace_bytes(S, d, D))
+        if n == 0:
+            raise ValueError("invalid sizes for lq_codebook_round")
+        workspace = torch.empty(n, dtype=torch.uint8, device=w.device)
+    _check(lib().lq_codebook_round(_dev(w, "w", (torch.float32,)), S,
+                                   _dev(M, "M", (torch.float32,)), d, D, int(mode),
+                                   _dev(b, "b", (torch.int8,)), _dev(mse, "mse", (torch.float64,)),
+                                   _dev(workspace, "workspace"),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)),
+           "lq_codebook_round")
+    return M, b, mse
 
 
 def check_wait_timeout(workspace, limit_ms=20, stream=None):

@@ -70,37 +70,49 @@ lq_status make_whiten(const lq_whiten_desc* T, int32_t K, lq::Whiten* out) {
 
 // Workspace layout of lq_gemm (byte offsets, all 256-aligned).
 struct WsLayout {
-  int path;          // 0: int8 tensor-core GEMV (batch <= 8); 1: fp32 GEMV over z;
-                     // 2: tcgen05 GEMM (batch >= lq::kTcMinBatch); 3: the int8 GEMV once per
-                     // group of gs tokens (when no single-launch plan fits)
+  int path;          // LQ_ROUTE_*: 0 int8 tensor-core GEMV (batch <= 8, two kernels); 1 no plan
+                     // fits; 2 tcgen05 GEMM (batch >= lq::kTcMinBatch); 3 the int8 GEMV once
+                     // per group of gs tokens (when no single-launch plan fits); 4 the
+                     // staged int8 GEMV (batch <= 8, one kernel); 5 the
+                     // dequantise-once GEMM (fp16 W, dense tcgen05 GEMM)
   size_t counters;   // uint32 completion counters of the split-K reduction
-  size_t z;          // path 0: prep output (fragments, weights, sums); path 1: float z [batch][L]
+  size_t z;          // paths 0/3: prep output (fragments, weights, sums); 2: fp16 z and token
+                     // scales; 4: fragments, token scales, chunk sums
   size_t partials;   // float [slices][batch][N]
   size_t total;
-  lq::GemvPlan gemv;
   lq::G8Plan g8;
+  lq::G8Plan g8g;    // path 3: the plan of a full group of gs tokens
   lq::G8Plan g8r;    // path 3: the plan of the last, smaller group
   int gs;            // path 3: tokens per group
   lq::TcPlan tc;
+  lq::BsPlan bs;
+  lq::DqPlan dq;
 };
 
-WsLayout layout_gemm(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D, int32_t Bh) {
+// The workspace layout of one lq_gemm call. `forced` >= 0 asks for that route (LQ_ROUTE_*),
+// which becomes LQ_ROUTE_NONE if its plan does not fit the shape; -1 chooses automatically.
+WsLayout layout_gemm(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D, int32_t Bh,
+                     int32_t forced = -1) {
   WsLayout w{};
   const int64_t L = lifted_bits(K, d, D);
   w.g8 = lq::plan_gemv_i8(batch, L, N, K, d, D, Bh);
   w.tc = lq::plan_gemm_tc(batch, L, N, K, d);
-  w.path = w.g8.ok ? 0 : (w.tc.ok && batch >= lq::kTcMinBatch ? 2 : 1);
-  // no single-launch GEMV fits: the largest token group whose int8 GEMV plan does, once per
-  // group
+  w.bs = lq::plan_gemv_bs(batch, L, N, K, d, D, Bh);
+  w.dq = lq::plan_gemm_dq(batch, N, K, d, D);
+  // token groups: the largest group whose int8 GEMV plan fits, once per group
+  bool groups_ok = false;
   for (int32_t gs : {8, 4, 2, 1}) {
-    if (w.path != 1 || gs >= batch) continue;
-    w.g8 = lq::plan_gemv_i8(gs, L, N, K, d, D, Bh);
-    w.g8r = batch % gs ? lq::plan_gemv_i8(batch % gs, L, N, K, d, D, Bh) : w.g8;
-    if (w.g8.ok && w.g8r.ok) {
-      w.path = 3;
+    if (gs >= batch) continue;
+    w.g8g = lq::plan_gemv_i8(gs, L, N, K, d, D, Bh);
+    w.g8r = batch % gs ? lq::plan_gemv_i8(batch % gs, L, N, K, d, D, Bh) : w.g8g;
+    if (w.g8g.ok && w.g8r.ok) {
       w.gs = gs;
+      groups_ok = true;
+      break;
     }
   }
+  w.path = w.g8.ok ? 0 : (w.tc.ok && batch >= lq::kTcMinBatch ? 2 : 1);
+  if (w.path == 1 && groups_ok) w.path = 3;
   // below kTcMinBatch tokens the tensor-core GEMM still wins once the groups are many: rough
   // B200 costs, each group streaming the codes at ~2 TB/s plus ~6 us, each wave of 128 x 256
   // tiles ~0.7 us per 64-coordinate stage
@@ -112,11 +124,33 @@ WsLayout layout_gemm(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D, 
     if (tc_s < gemv_s) w.path = 2;
   }
   if (w.path == 1 && w.tc.ok && batch > 8) w.path = 2;
+  // the staged GEMV serves batches the two-kernel GEMV cannot take in one launch
+  if (w.bs.ok && w.path != 0) w.path = 4;
+  // the tensor-core routes: the lifted GEMM contracts over L coordinates; the dequantise-once
+  // GEMM over G*d inputs (D/d times fewer MMA flops) after writing and reading fp16 W once.
+  // Rough B200 costs: ~1.0 PFLOP/s lifted, ~1.3 PFLOP/s dense, ~5 TB/s for W's two passes.
+  if (w.path == 2 && w.dq.ok) {
+    const double tc_s = 2.0 * batch * (double)N * (double)L / 1.0e15;
+    const double dq_s = 2.0 * batch * (double)N * (double)w.dq.Kw / 1.3e15 +
+                        2.0 * (double)w.dq.w_bytes / 5.0e12 + 10e-6;
+    if (dq_s < tc_s) w.path = 5;
+  }
+  if (forced >= 0) {
+    const bool fits = forced == 0 ? w.g8.ok : forced == 2 ? w.tc.ok : forced == 3 ? groups_ok
+                    : forced == 4 ? w.bs.ok : forced == 5 ? w.dq.ok : false;
+    w.path = fits ? forced : 1;
+  }
   size_t ncounters = 0, npartials = 0, nz = 0;
-  if (w.path == 3) {
+  if (w.path == 5) {
+    nz = (w.dq.w_bytes + w.dq.x_bytes + w.dq.scale_bytes + 3) / 4;
+  } else if (w.path == 4) {
+    ncounters = (size_t)w.bs.R;
+    nz = (w.bs.sumz_bytes + 3) / 4;   // per-slice sums of z
+    npartials = w.bs.gacc_bytes / 4;  // int32 totals
+  } else if (w.path == 3) {
     // the groups run one after the other on the stream and share the scratch
-    for (const lq::G8Plan* g : {&w.g8, &w.g8r}) {
-      const int nb = g == &w.g8 ? w.gs : (batch % w.gs ? batch % w.gs : w.gs);
+    for (const lq::G8Plan* g : {&w.g8g, &w.g8r}) {
+      const int nb = g == &w.g8g ? w.gs : (batch % w.gs ? batch % w.gs : w.gs);
       ncounters = std::max(ncounters, (size_t)g->R);
       npartials = std::max(npartials, g->S > 1 ? (size_t)g->S * nb * N : (size_t)0);
       nz = std::max(nz, (g->frag_bytes + g->wtab_bytes + g->csum_bytes + 3) / 4);
@@ -127,11 +161,6 @@ WsLayout layout_gemm(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D, 
     ncounters = (size_t)w.g8.R;
     npartials = w.g8.S > 1 ? (size_t)w.g8.S * batch * N : 0;
     nz = (w.g8.frag_bytes + w.g8.wtab_bytes + w.g8.csum_bytes + 3) / 4;   // prep output
-  } else {
-    w.gemv = lq::plan_gemv(batch, L, N);
-    ncounters = (size_t)w.gemv.ntg * w.gemv.ntiles;
-    npartials = w.gemv.nsl > 1 ? (size_t)w.gemv.nsl * batch * N : 0;
-    nz = (size_t)batch * L;
   }
   size_t off = sizeof(lq::WsHeader);
   w.counters = off;
@@ -286,14 +315,29 @@ int32_t lq_gemm_launches(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t
   if (!valid_code(K, d, D) || batch < 1 || batch > kMaxBatch || N < 1 || K > kMaxK) return 0;
   if (block < 0 || block > LQ_MAX_HADAMARD || (block & (block - 1)) != 0) return 0;
   const WsLayout lay = layout_gemm(batch, K, N, d, D, block);
-  // every path: a prologue kernel and a contraction kernel, per token group on path 3
+  // path 4: one kernel; paths 0 and 2: a prologue kernel and a contraction kernel, per token
+  // group on path 3; path 1: nothing (the call is rejected)
+  if (lay.path == 4) return 1;
+  if (lay.path == 1) return 0;
+  if (lay.path == 5) return 3;   // W, xt, GEMM
   return lay.path == 3 ? 2 * ((batch + lay.gs - 1) / lay.gs) : 2;
 }
 
-lq_status lq_gemm(const void* x, lq_dtype xdt, int32_t batch, const lq_whiten_desc* T,
-                  const uint32_t* packed, const float* M, const void* s, lq_dtype sdt,
-                  int32_t d, int32_t D, int32_t K, int32_t N, float* y, void* workspace,
-                  size_t workspace_bytes, lq_stream stream) {
+int32_t lq_gemm_route(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D,
+                      int32_t block) {
+  if (!valid_code(K, d, D) || batch < 1 || batch > kMaxBatch || N < 1 || K > kMaxK) return -1;
+  if (block < 0 || block > LQ_MAX_HADAMARD || (block & (block - 1)) != 0) return -1;
+  return layout_gemm(batch, K, N, d, D, block).path;
+}
+
+}  // extern "C"
+
+namespace {
+
+lq_status gemm_impl(const void* x, lq_dtype xdt, int32_t batch, const lq_whiten_desc* T,
+                    const uint32_t* packed, const float* M, const void* s, lq_dtype sdt,
+                    int32_t d, int32_t D, int32_t K, int32_t N, float* y, void* workspace,
+                    size_t workspace_bytes, lq_stream stream, int32_t forced) {
   clear_error();
   if (!valid_code(K, d, D)) return fail(LQ_EINVAL, "invalid code sizes K=%d d=%d D=%d", K, d, D);
   if (batch < 1 || batch > kMaxBatch) return fail(LQ_EINVAL, "batch = %d out of range", batch);
@@ -309,7 +353,7 @@ lq_status lq_gemm(const void* x, lq_dtype xdt, int32_t batch, const lq_whiten_de
   lq::Whiten w;
   lq_status st = make_whiten(T, K, &w);
   if (st != LQ_OK) return st;
-  const WsLayout lay = layout_gemm(batch, K, N, d, D, w.block);
+  const WsLayout lay = layout_gemm(batch, K, N, d, D, w.block, forced);
   if (workspace_bytes < lay.total)
     return fail(LQ_EINVAL, "workspace of %zu bytes is smaller than the %zu bytes needed",
                 workspace_bytes, lay.total);
@@ -318,6 +362,22 @@ lq_status lq_gemm(const void* x, lq_dtype xdt, int32_t batch, const lq_whiten_de
   const int64_t L = lifted_bits(K, d, D);
   uint32_t* counters = reinterpret_cast<uint32_t*>(ws + lay.counters);
   float* partials = reinterpret_cast<float*>(ws + lay.partials);
+  if (lay.path == 4) {
+    lq::BsScratch sc{};
+    sc.sumz = reinterpret_cast<float*>(ws + lay.z);
+    sc.gacc = reinterpret_cast<int*>(ws + lay.partials);
+    sc.counters = counters;
+    sc.status = reinterpret_cast<uint32_t*>(ws);
+    cudaError_t e = lq::launch_gemv_bs(lay.bs, x, (int)xdt, batch, K, w, M, d, D, L, packed,
+                                       row_stride_bytes(K, d, D), N, s, (int)sdt, y, sc, cs);
+    return e == cudaSuccess ? LQ_OK : cuda_fail(e, "lq_gemm (staged gemv)");
+  }
+  if (lay.path == 5) {
+    cudaError_t e = lq::launch_gemm_dq(lay.dq, x, (int)xdt, batch, K, w, M, d, D, packed,
+                                       row_stride_bytes(K, d, D), N, s, (int)sdt, y, ws + lay.z,
+                                       reinterpret_cast<uint32_t*>(ws), cs);
+    return e == cudaSuccess ? LQ_OK : cuda_fail(e, "lq_gemm (dequantise-once gemm)");
+  }
   if (lay.path == 2) {
     cudaError_t e = lq::launch_gemm_tc(lay.tc, x, (int)xdt, batch, K, w, M, d, D, L, packed,
                                        row_stride_bytes(K, d, D), N, s, (int)sdt, y, ws + lay.z,
@@ -334,22 +394,114 @@ lq_status lq_gemm(const void* x, lq_dtype xdt, int32_t batch, const lq_whiten_de
     for (int32_t t0 = 0; t0 < batch; t0 += lay.gs) {
       const int32_t nb = std::min<int32_t>(lay.gs, batch - t0);
       const char* xt = static_cast<const char*>(x) + (size_t)t0 * K * dtype_size(xdt);
-      cudaError_t e = lq::launch_gemv_i8(nb == lay.gs ? lay.g8 : lay.g8r, xt, (int)xdt, nb, K, w, M, d,
+      cudaError_t e = lq::launch_gemv_i8(nb == lay.gs ? lay.g8g : lay.g8r, xt, (int)xdt, nb, K, w, M, d,
                                          D, L, packed, row_stride_bytes(K, d, D), N, s, (int)sdt,
                                          y + (size_t)t0 * N, ws + lay.z, partials, counters, cs);
       if (e != cudaSuccess) return cuda_fail(e, "lq_gemm (int8 gemv, token group)");
     }
     return LQ_OK;
   }
-  if (lay.gemv.ntiles > 65535 || lay.gemv.ntg > 65535)
-    return fail(LQ_EUNSUPPORTED, "N or batch too large for one launch");
-  float* z = reinterpret_cast<float*>(ws + lay.z);
-  cudaError_t e = lq::launch_lift_f32(x, (int)xdt, batch, K, w, M, d, D, z, counters,
-                                      lay.gemv.ntg * lay.gemv.ntiles, cs);
-  if (e != cudaSuccess) return cuda_fail(e, "lq_gemm (lift)");
-  e = lq::launch_gemv(lay.gemv, z, L, batch, packed, row_stride_bytes(K, d, D) / 4, N, s,
-                      (int)sdt, y, partials, counters, cs);
-  return e == cudaSuccess ? LQ_OK : cuda_fail(e, "lq_gemm (gemv)");
+  return fail(LQ_EUNSUPPORTED, "no GEMV or GEMM plan fits batch=%d K=%d N=%d d=%d D=%d block=%d%s",
+              batch, K, N, d, D, w.block, forced >= 0 ? " on the requested route" : "");
+}
+
+}  // namespace
+
+extern "C" {
+
+lq_status lq_gemm(const void* x, lq_dtype xdt, int32_t batch, const lq_whiten_desc* T,
+                  const uint32_t* packed, const float* M, const void* s, lq_dtype sdt,
+                  int32_t d, int32_t D, int32_t K, int32_t N, float* y, void* workspace,
+                  size_t workspace_bytes, lq_stream stream) {
+  return gemm_impl(x, xdt, batch, T, packed, M, s, sdt, d, D, K, N, y, workspace,
+                   workspace_bytes, stream, -1);
+}
+
+lq_status lq_gemm_on_route(const void* x, lq_dtype xdt, int32_t batch, const lq_whiten_desc* T,
+                           const uint32_t* packed, const float* M, const void* s, lq_dtype sdt,
+                           int32_t d, int32_t D, int32_t K, int32_t N, float* y,
+                           void* workspace, size_t workspace_bytes, int32_t route,
+                           lq_stream stream) {
+  clear_error();
+  if (route < 0 || route > LQ_ROUTE_GEMM_DQ || route == LQ_ROUTE_NONE)
+    return fail(LQ_EINVAL, "unknown route %d", route);
+  return gemm_impl(x, xdt, batch, T, packed, M, s, sdt, d, D, K, N, y, workspace,
+                   workspace_bytes, stream, route);
+}
+
+size_t lq_gemm_route_workspace_bytes(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D,
+                                     int32_t block, int32_t route) {
+  if (!valid_code(K, d, D) || batch < 1 || batch > kMaxBatch || N < 1 || K > kMaxK) return 0;
+  if (block < 0 || block > LQ_MAX_HADAMARD || (block & (block - 1)) != 0) return 0;
+  if (route < 0 || route > LQ_ROUTE_GEMM_DQ || route == LQ_ROUTE_NONE) return 0;
+  const WsLayout lay = layout_gemm(batch, K, N, d, D, block, route);
+  return lay.path == route ? lay.total : 0;
+}
+
+namespace {
+
+struct CbLayout {
+  size_t b, err, pA, pC, pE, total;
+};
+
+CbLayout layout_codebook(int64_t S, int32_t d, int32_t D, bool own_codes) {
+  CbLayout l{};
+  const size_t parts = lq::codebook_partials(S);
+  size_t off = sizeof(lq::WsHeader);
+  l.b = off;
+  if (own_codes) off = round_up(off + (size_t)S * D, 256);
+  l.err = off;
+  off = round_up(off + (size_t)S * sizeof(float), 256);
+  l.pA = off;
+  off = round_up(off + parts * d * D * sizeof(double), 256);
+  l.pC = off;
+  off = round_up(off + parts * D * D * sizeof(long long), 256);
+  l.pE = off;
+  off = round_up(off + parts * sizeof(double), 256);
+  l.total = off;
+  return l;
+}
+
+lq_status check_codebook(int64_t S, int32_t d, int32_t D, int32_t mode) {
+  if (S < 1 || S > ((int64_t)1 << 31)) return fail(LQ_EINVAL, "S = %lld out of range", (long long)S);
+  if (d < 1 || D < d || D > LQ_MAX_D) return fail(LQ_EINVAL, "invalid code sizes d=%d D=%d", d, D);
+  if (mode != LQ_ENCODE_EXACT && mode != LQ_ENCODE_SEEDED)
+    return fail(LQ_EINVAL, "unknown encode mode %d", mode);
+  if (d > 16) return fail(LQ_EUNSUPPORTED, "lq_codebook_round: d = %d > 16", d);
+  if (mode == LQ_ENCODE_EXACT && D > 24)
+    return fail(LQ_EUNSUPPORTED, "lq_codebook_round: exact search with D = %d > 24", D);
+  if (mode == LQ_ENCODE_SEEDED && D - d > 24)
+    return fail(LQ_EUNSUPPORTED, "lq_codebook_round: seeded search with D - d = %d > 24", D - d);
+  return LQ_OK;
+}
+
+}  // namespace
+
+size_t lq_codebook_workspace_bytes(int64_t S, int32_t d, int32_t D) {
+  if (S < 1 || S > ((int64_t)1 << 31) || d < 1 || D < d || D > LQ_MAX_D) return 0;
+  return layout_codebook(S, d, D, true).total;
+}
+
+lq_status lq_codebook_round(const float* w, int64_t S, float* M, int32_t d, int32_t D,
+                            int32_t mode, int8_t* b_out, double* mse, void* workspace,
+                            size_t workspace_bytes, lq_stream stream) {
+  clear_error();
+  lq_status st = check_codebook(S, d, D, mode);
+  if (st != LQ_OK) return st;
+  if (!w || !M || !workspace) return fail(LQ_EINVAL, "null pointer");
+  if (!aligned(w, 4) || !aligned(M, 4) || !aligned(workspace, 256) || (mse && !aligned(mse, 8)))
+    return fail(LQ_EINVAL, "misaligned w/M/workspace/mse");
+  const CbLayout l = layout_codebook(S, d, D, b_out == nullptr);
+  if (workspace_bytes < l.total)
+    return fail(LQ_EINVAL, "workspace of %zu bytes is smaller than the %zu bytes needed",
+                workspace_bytes, l.total);
+  char* ws = static_cast<char*>(workspace);
+  int8_t* b = b_out ? b_out : reinterpret_cast<int8_t*>(ws + l.b);
+  cudaError_t e = lq::launch_codebook_round(
+      w, S, M, d, D, mode, b, reinterpret_cast<float*>(ws + l.err),
+      reinterpret_cast<double*>(ws + l.pA), reinterpret_cast<long long*>(ws + l.pC),
+      reinterpret_cast<double*>(ws + l.pE), mse, (cudaStream_t)stream);
+  return e == cudaSuccess ? LQ_OK : cuda_fail(e, "lq_codebook_round");
 }
 
 lq_status lq_device_status(void* workspace, int32_t* code, lq_stream stream) {

@@ -10,7 +10,9 @@
 //    2^e chosen from a bound on |z|, written as fp16 z * 2^e. Inside every 32-coordinate word
 //    the coordinates are stored in the order q0, q0+16, q0+1, q0+17, ..., q0+15, q0+31 -- the
 //    order in which the GEMM unpacks a 32-bit code word into fp16 pairs (see pm1_pair).
-//  * gemm_tc_kernel (persistent, one CTA per SM): 128-token x 256-row output tiles. A warp
+//  * gemm_tc_kernel (persistent, one CTA per SM): 128-token x 256-row output tiles, taken
+//    token tile fastest, so that the CTAs of one wave share the codes of a few row tiles in L2
+//    while the (smaller) z matrix stays resident there. A warp
 //    loads the fp16 z tile with TMA (128-byte swizzle); eight warps expand the stored bits of
 //    256 rows into +-1 fp16 in the same swizzled K-major layout; one thread issues
 //    tcgen05.mma (fp32 accumulation in tensor memory, two accumulators so the epilogue of one
@@ -71,7 +73,7 @@ struct TcArgs {
   const void* s;
   float* y;
   uint32_t* status;         // workspace status word
-  int N, batch, nks, tiles_n, tiles, sdt, vec_store;
+  int N, batch, nks, tiles_n, tiles_m, tiles, sdt, vec_store;
 };
 
 __device__ __forceinline__ uint64_t globaltimer() {
@@ -158,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- epilogue
     int lt = 0;
     for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x, ++lt) {
-      const int tn = tile % a.tiles_n, tm = tile / a.tiles_n;
+      const int tm = tile % a.tiles_m, tn = tile / a.tiles_m;
       const int b = lt & 1;
       // tcgen05.ld below is warp-collective: every lane must take the same branch here
       if (!__all_sync(0xffffffffu, wait_phase(&ctl->tmem_full[b], (lt >> 1) & 1, abort, true))) {
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t ctr = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < a.tiles; tile += gridDim.x) {
-        const int tm = tile / a.tiles_n;
+        const int tm = tile % a.tiles_m;
         for (int k = 0; k < a.nks; ++k, ++ctr) {
           const int slot = ctr % NSTAGE;
           if (!wait_phase(&ctl->empty[slot], ((ctr / NSTAGE) & 1) ^ 1, abort, true)) {
@@ -274,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ctr = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < a.tiles; tile += gridDim.x) {
-      const int tn = tile % a.tiles_n;
+      const int tn = tile / a.tiles_m;
       const int n = tn * BN + p;
       const bool valid = n < a.N;
       const uint2* rp = reinterpret_cast<const uint2*>(a.packed + (valid ? (int64_t)n * a.row_words : 0));
@@ -473,6 +475,9 @@ int sm_count() {
 
 }  // namespace tc
 
+TensorMapEncodeFn tensor_map_encode_fn() { return tc::encode_fn(); }
+int tc_sm_count() { return tc::sm_count(); }
+
 TcPlan plan_gemm_tc(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d) {
   TcPlan p{};
   if (batch < 1) return p;
@@ -539,6 +544,7 @@ cudaError_t launch_gemm_tc(const TcPlan& pl, const void* x, int xdt, int32_t bat
   a.batch = batch;
   a.nks = pl.nks;
   a.tiles_n = pl.tiles_n;
+  a.tiles_m = pl.tiles_m;
   a.tiles = pl.tiles;
   a.sdt = sdt;
   a.vec_store = (N % 4 == 0) && (reinterpret_cast<uintptr_t>(y) % 16 == 0);

@@ -1,6 +1,7 @@
 // lq_internal.cuh -- declarations shared by the liblq CUDA sources (not part of the ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -55,22 +56,6 @@ cudaError_t launch_lift_f32(const void* x, int xdt, int32_t batch, int32_t K, Wh
                             const float* M, int32_t d, int32_t D, float* z, uint32_t* zero_ptr,
                             int32_t zero_words, cudaStream_t st);
 
-// Plan of the small-batch GEMV over z (fp32, in global memory).
-struct GemvPlan {
-  int tb;        // tokens per CTA
-  int ntg;       // token groups
-  int sw;        // 32-bit words of a row per K-slice
-  int nsl;       // K-slices
-  int rt;        // rows per CTA
-  int ntiles;    // row tiles
-  size_t smem;   // dynamic shared memory per CTA
-};
-GemvPlan plan_gemv(int32_t batch, int64_t L, int32_t N);
-cudaError_t launch_gemv(const GemvPlan& p, const float* z, int64_t L, int32_t batch,
-                        const uint32_t* packed, int64_t row_words, int32_t N, const void* s,
-                        int sdt, float* y, float* partials, uint32_t* counters,
-                        cudaStream_t st);
-
 // Plan of the int8 tensor-core GEMV (batch <= 8): a prep kernel per 512-bit chunk, then
 // S K-slices x R row ranges, one CTA each.
 struct G8Plan {
@@ -120,9 +105,88 @@ cudaError_t launch_gemm_tc(const TcPlan& pl, const void* x, int xdt, int32_t bat
                            const uint32_t* packed, int64_t row_bytes, int32_t N, const void* s,
                            int sdt, float* y, void* scratch, uint32_t* status, cudaStream_t st);
 
+// Plan of the staged int8 tensor-core GEMV (batch <= 8): one launch of S K-slices x R row
+// ranges, one CTA per SM; each CTA builds its slice's activation operand itself.
+struct BsPlan {
+  bool ok;
+  int nt;             // 8-column MMA tiles (2 tokens each)
+  int nchunk;         // 512-bit chunks per row
+  int sc;             // chunks per slice
+  int S;              // slices
+  int R;              // row ranges
+  int rq, rrem;       // rows per range: rq + (range < rrem)
+  int rows_max;       // rq + 1
+  int wch;            // chunks per stage window
+  int stride;         // shared-memory row stride of a stage
+  int NS;             // ring stages
+  int nctas;          // S * R
+  int xs_floats;      // whitened inputs of a slice, per token
+  size_t smem;        // dynamic shared memory per CTA
+  size_t frag_smem;   // shared memory: the slice's fragments
+  size_t prep_smem;   // shared memory: whitening, z and M scratch
+  size_t sumz_bytes;  // scratch: per-slice sums of z [S][batch] (S > 1)
+  size_t gacc_bytes;  // scratch: int32 totals [batch][N][4] (S > 1), zero at rest
+};
+BsPlan plan_gemv_bs(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, int32_t D,
+                    int32_t Bh);
+// Global scratch of one call (used when S > 1): gacc and counters [R] must be zero before the
+// first call and are left zero by every call; sumz is rewritten by every call.
+struct BsScratch {
+  float* sumz;
+  int* gacc;
+  uint32_t* counters;
+  uint32_t* status;
+};
+cudaError_t launch_gemv_bs(const BsPlan& pl, const void* x, int xdt, int32_t batch, int32_t K,
+                           Whiten T, const float* M, int32_t d, int32_t D, int64_t L,
+                           const uint32_t* packed, int64_t row_bytes, int32_t N, const void* s,
+                           int sdt, float* y, const BsScratch& ws, cudaStream_t st);
+
+// Plan of the dequantise-once GEMM (large batches): W = blockwise M b in fp16 [N][Kw], fp16
+// T(x) [batch][Kw] with a per-token power of two, then a persistent tcgen05 GEMM over
+// 128-token x 256-row tiles.
+struct DqPlan {
+  bool ok;
+  int G;               // blocks of d inputs per row
+  int Kw;              // G*d padded to the 64-input stage
+  int nks;             // stages per tile
+  int tiles_n, tiles_m, tiles;
+  size_t smem;         // GEMM dynamic shared memory per CTA
+  size_t xt_smem;      // xt kernel dynamic shared memory
+  size_t dq_smem;      // dequantisation kernel dynamic shared memory per CTA
+  int dq_ctas_per_sm;  // dequantisation CTAs per SM
+  size_t w_bytes;      // scratch: fp16 W [N][Kw]
+  size_t x_bytes;      // scratch: fp16 xt [batch][Kw], after W
+  size_t scale_bytes;  // scratch: float 2^-e [batch], after xt
+};
+DqPlan plan_gemm_dq(int32_t batch, int32_t N, int32_t K, int32_t d, int32_t D);
+// scratch: w_bytes + x_bytes + scale_bytes bytes, 256-byte aligned; status: workspace word
+cudaError_t launch_gemm_dq(const DqPlan& pl, const void* x, int xdt, int32_t batch, int32_t K,
+                           Whiten T, const float* M, int32_t d, int32_t D,
+                           const uint32_t* packed, int64_t row_bytes, int32_t N, const void* s,
+                           int sdt, float* y, void* scratch, uint32_t* status, cudaStream_t st);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (nullptr if unavailable),
+// and the SM count of the current device (0 on error); both cached.
+typedef CUresult (*TensorMapEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                      const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                      const cuuint32_t*, CUtensorMapInterleave,
+                                      CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                      CUtensorMapFloatOOBfill);
+TensorMapEncodeFn tensor_map_encode_fn();
+int tc_sm_count();
+
 // Nearest-codeword encoding, block by block: b [N][ceil(K/d)][D] +1/-1, err [N][G] or null.
 // mode 0: all 2^D codewords; mode 1: first d coordinates solved, the rest enumerated.
 cudaError_t launch_encode(const float* w, int64_t N, int32_t K, const float* M, int32_t d,
                           int32_t D, int32_t mode, int8_t* b, float* err, cudaStream_t st);
+
+// One round of the codebook fit (see lq_codebook.cu): the encoder into b [S][D] and err [S],
+// then the sums into the partials (codebook_partials(S) CTAs: pA [parts][d*D], pC
+// [parts][D*D], pE [parts]) and the solve into M and *mse (mse may be null).
+size_t codebook_partials(int64_t S);
+cudaError_t launch_codebook_round(const float* w, int64_t S, float* M, int32_t d, int32_t D,
+                                  int32_t mode, int8_t* b, float* err, double* pA, long long* pC,
+                                  double* pE, double* mse, cudaStream_t st);
 
 }  // namespace lq

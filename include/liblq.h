@@ -150,6 +150,26 @@ LQ_API size_t lq_gemm_workspace_bytes(int32_t batch, int32_t K, int32_t N, int32
 LQ_API int32_t lq_gemm_launches(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D,
                                 int32_t block);
 
+/* Which kernels lq_gemm runs for this shape and Hadamard block (-1 on invalid sizes). Host-only,
+ * touches no device. No counterpart on the pages: it lets tests and profiles name the path.
+ *   LQ_ROUTE_GEMV_I8     int8 tensor-core GEMV over bit planes, prologue + contraction kernels
+ *   LQ_ROUTE_NONE        no plan fits the shape: lq_gemm returns LQ_EUNSUPPORTED
+ *   LQ_ROUTE_GEMM_TC     tcgen05 tensor-core GEMM over fp16 z (batch >= 64, or where cheaper)
+ *   LQ_ROUTE_GEMV_GROUPS LQ_ROUTE_GEMV_I8 once per group of tokens
+ *   LQ_ROUTE_GEMV_BULK   int8 tensor-core GEMV with bulk-copied code rows, one cooperative
+ *                        kernel (batch <= 8 where its plan fits)
+ *   LQ_ROUTE_GEMM_DQ     W = blockwise M b dequantised once to fp16 in the workspace, then a
+ *                        dense tcgen05 GEMM of fp16 T(x) against W (large batches, where its
+ *                        D/d-times smaller contraction outweighs writing and reading W) */
+#define LQ_ROUTE_GEMV_I8 0
+#define LQ_ROUTE_NONE 1
+#define LQ_ROUTE_GEMM_TC 2
+#define LQ_ROUTE_GEMV_GROUPS 3
+#define LQ_ROUTE_GEMV_BULK 4
+#define LQ_ROUTE_GEMM_DQ 5
+LQ_API int32_t lq_gemm_route(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D,
+                             int32_t block);
+
 /* The decode operator, y = s . (W T(x)) (paper sec. 3 intro: o = diag(s) W (M T a);
  * review: diag(s) W_q (T* a)).
  *   x       [batch][K] of dtype xdt (f32, f16 or bf16)
@@ -157,13 +177,32 @@ LQ_API int32_t lq_gemm_launches(int32_t batch, int32_t K, int32_t N, int32_t d, 
  *   M       [d][D] float32;  s [N] of dtype sdt;  y [batch][N] float32 (overwritten)
  *   workspace: lq_gemm_workspace_bytes(...) bytes, 256-byte aligned, caller-owned.
  *     It must be zero-filled before its first use; every call leaves it ready for the next.
- * Accumulation is fp32 in a fixed order: the result does not depend on timing.
+ * Accumulation is exact in int32 (the GEMV routes add integer products of int8 planes of z) or
+ * fp32 in a fixed order (tensor-core GEMM): the result does not depend on timing.
  * Errors: LQ_EINVAL (null or misaligned pointers, batch < 1, N < 1, bad sizes,
- * workspace too small), LQ_EUNSUPPORTED (block > LQ_MAX_HADAMARD), LQ_ECUDA. */
+ * workspace too small), LQ_EUNSUPPORTED (block > LQ_MAX_HADAMARD, or a shape that no kernel
+ * plan fits: lq_gemm_route reports LQ_ROUTE_NONE), LQ_ECUDA. */
 LQ_API lq_status lq_gemm(const void* x, lq_dtype xdt, int32_t batch, const lq_whiten_desc* T,
                   const uint32_t* packed, const float* M, const void* s, lq_dtype sdt,
                   int32_t d, int32_t D, int32_t K, int32_t N, float* y, void* workspace,
                   size_t workspace_bytes, lq_stream stream);
+
+/* lq_gemm on a chosen route (LQ_ROUTE_GEMV_I8, _GEMM_TC, _GEMV_GROUPS, _GEMV_BULK or _GEMM_DQ)
+ * instead of the one lq_gemm_route picks: the same operator and arguments, for comparing the
+ * kernel families on one shape (both large-batch GEMMs, for instance). No counterpart on the
+ * pages. The workspace must hold lq_gemm_route_workspace_bytes(..., route) bytes, zero-filled
+ * before its first use. Errors: as lq_gemm, plus LQ_EINVAL for an unknown route and
+ * LQ_EUNSUPPORTED when the route's plan does not fit the shape. */
+LQ_API lq_status lq_gemm_on_route(const void* x, lq_dtype xdt, int32_t batch,
+                                  const lq_whiten_desc* T, const uint32_t* packed,
+                                  const float* M, const void* s, lq_dtype sdt, int32_t d,
+                                  int32_t D, int32_t K, int32_t N, float* y, void* workspace,
+                                  size_t workspace_bytes, int32_t route, lq_stream stream);
+
+/* Workspace bytes of lq_gemm_on_route for this shape, Hadamard block and route; 0 on invalid
+ * sizes or when the route's plan does not fit. */
+LQ_API size_t lq_gemm_route_workspace_bytes(int32_t batch, int32_t K, int32_t N, int32_t d,
+                                            int32_t D, int32_t block, int32_t route);
 
 /* Bytes of the scratch array that lq_gemm_noalloc keeps on every device that loads the library. */
 #define LQ_NOALLOC_SCRATCH_BYTES (8u << 20)
@@ -174,9 +213,11 @@ LQ_API lq_status lq_gemm(const void* x, lq_dtype xdt, int32_t batch, const lq_wh
  * framework or allocator they cannot call into (a plugin, an inference-server backend with a
  * fixed budget), or they run where allocating is not allowed. This entry point takes the same
  * arguments as lq_gemm except the workspace, allocates nothing (no cudaMalloc, no cudaFree, no
- * allocating library routine) and keeps its scratch (split-K counters and slice partials) in a
- * fixed device array of LQ_NOALLOC_SCRATCH_BYTES bytes that every GPU which loads the library
- * holds until the process exits.
+ * allocating library routine) and keeps its scratch in a fixed device array of
+ * LQ_NOALLOC_SCRATCH_BYTES bytes that every GPU which loads the library holds until the process
+ * exits. The array holds what lq_gemm keeps in its workspace on this path: the prologue's int8
+ * activation fragments (most of it for large K), their per-chunk column weights and sums of z,
+ * the split-K completion counters and the fp32 slice partials.
  *   - batch 1..8 (the small-batch GEMV); shapes whose scratch would exceed
  *     LQ_NOALLOC_SCRATCH_BYTES are rejected with LQ_EINVAL and a reason in lq_last_error().
  *   - The first call on a device sets that device up (finds the array's device address and
@@ -193,6 +234,30 @@ LQ_API lq_status lq_gemm_noalloc(const void* x, lq_dtype xdt, int32_t batch,
                                  const lq_whiten_desc* T, const uint32_t* packed, const float* M,
                                  const void* s, lq_dtype sdt, int32_t d, int32_t D, int32_t K,
                                  int32_t N, float* y, lq_stream stream);
+
+/* Workspace bytes of lq_codebook_round for S samples (0 on invalid sizes). */
+LQ_API size_t lq_codebook_workspace_bytes(int64_t S, int32_t d, int32_t D);
+
+/* One round of the offline codebook fit (review "Method": M is fitted to a standard Gaussian;
+ * paper sec. 3.1, Eq. (1): M* = argmin E ||w - M b*(w)||^2, its text cut before the gradient
+ * path). Reading: alternating minimisation over samples w_s:
+ *   (1) b_s = the nearest codeword of w_s under M (lq_encode's search, `mode` as there);
+ *   (2) M = (sum_s w_s b_s^T)(sum_s b_s b_s^T)^-1, the least-squares fit with the codes fixed
+ *       (where the straight-through gradient -2 sum_s (w_s - M b_s) b_s^T vanishes).
+ *   w      [S][d] fp32 device (the samples, e.g. N(0, 1) draws).
+ *   M      [d][D] fp32 device: read by step (1), overwritten by step (2) unless sum b b^T is
+ *          singular, in which case it is left unchanged and *mse is -1.
+ *   b_out  [S][D] int8 device (+1/-1 codes of step (1)) or NULL (the workspace holds them).
+ *   mse    one fp64 on the device or NULL: sum_s ||w_s - M b_s||^2 / (S d) of step (1) (the
+ *          encoder's fp32 distances added in fp64).
+ *   workspace: lq_codebook_workspace_bytes(S, d, D) bytes, 256-byte aligned, caller-owned.
+ * The sums run in fp64 (sum w b^T) and exactly in int64 (sum b b^T) in a fixed order, the solve
+ * in fp64 with partial pivoting: the result does not depend on timing. Asynchronous on
+ * `stream`. Errors: LQ_EINVAL (null or misaligned pointers, S < 1, bad sizes, unknown mode,
+ * workspace too small), LQ_EUNSUPPORTED (as lq_encode), LQ_ECUDA. */
+LQ_API lq_status lq_codebook_round(const float* w, int64_t S, float* M, int32_t d, int32_t D,
+                                   int32_t mode, int8_t* b_out, double* mse, void* workspace,
+                                   size_t workspace_bytes, lq_stream stream);
 
 /* Synchronise `stream`, then read the workspace status word into *code (0 = no device-side
  * failure) and clear it. Returns LQ_OK, or the lq_status that the word records. */

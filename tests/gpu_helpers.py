@@ -1,5 +1,7 @@
 """Helpers shared by the GPU parity tests: move synthetic layers to the device and compare
 results with the oracle's."""
+import os
+
 import numpy as np
 import torch
 
@@ -41,14 +43,16 @@ def device_layer(layer, dev="cuda"):
     )
 
 
-def run_gemm(layer, dl, workspace=None):
+def run_gemm(layer, dl, workspace=None, route=None):
     return lq.gemm(dl["x"], dl["packed"], dl["M"], dl["s"], layer.d, layer.D, sign=dl["sign"],
-                   block=layer.block, workspace=workspace)
+                   block=layer.block, workspace=workspace, route=route)
 
 
-def oracle_rows(orc, layer, rows, tokens=None, nthreads=8):
+def oracle_rows(orc, layer, rows, tokens=None, nthreads=None):
     """Oracle outputs for a subset of rows (and tokens): [len(tokens)][len(rows)] fp64."""
     x = layer.x if tokens is None else layer.x[tokens]
+    if nthreads is None:
+        nthreads = max(1, len(os.sched_getaffinity(0)))
     p = orc.pack(layer.b[rows], layer.K, layer.d, layer.D)
     return orc.forward(x, p, layer.M, layer.s[rows], layer.d, layer.D, sign=layer.sign,
                        block=layer.block, nthreads=nthreads)

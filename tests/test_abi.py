@@ -88,8 +88,10 @@ def test_wait_timeout_check_arguments_without_gpu(L):
 
 
 def test_gemm_launches(L):
-    assert lq.gemm_launches(1, 4096, 4096, 10, 24, 256) == 2        # int8 GEMV
-    assert lq.gemm_launches(2048, 8192, 28672, 10, 24, 256) == 2    # tcgen05 GEMM
+    assert lq.gemm_launches(1, 4096, 4096, 10, 24, 256) == 2        # two-kernel int8 GEMV
+    assert lq.gemm_launches(2, 8192, 300, 10, 24, 4096) == 2        # two-kernel int8 GEMV
+    assert lq.gemm_launches(2048, 8192, 28672, 10, 24, 256) == 3    # W, xt, dense GEMM
+    assert lq.gemm_launches(64, 8192, 28672, 10, 24, 256) == 2      # lifted tcgen05 GEMM
     n16 = lq.gemm_launches(16, 28672, 8192, 10, 24, 256)            # token groups
     assert n16 >= 4 and n16 % 2 == 0
     assert lq.gemm_launches(0, 4096, 4096, 10, 24, 256) == 0
@@ -100,18 +102,33 @@ def test_gemm_launches(L):
                                             (28672, 8192, 4), (256, 128, 8), (40, 64, 8)])
 def test_small_batches_run_as_one_gemv(L, K, N, max_single):
     """Up to 4 tokens on the Llama-3-70B MLP shapes, up to 8 on 4096- and 8192-wide layers, the
-    int8 GEMV runs once (prep + contraction): the slices widen until a CTA's rows fit its warps'
-    partial slots instead of splitting the batch into token groups."""
+    batch runs as one int8 GEMV (one bulk-staged kernel, or prep + contraction) instead of
+    token groups."""
     for b in range(1, max_single + 1):
-        assert lq.gemm_launches(b, K, N, 10, 24, 256) == 2, b
+        route = lq.gemm_route(b, K, N, 10, 24, 256)
+        assert route in (lq.ROUTE_GEMV_BULK, lq.ROUTE_GEMV_I8), (b, route)
+        assert lq.gemm_launches(b, K, N, 10, 24, 256) == (1 if route == lq.ROUTE_GEMV_BULK else 2)
 
 
 @pytest.mark.parametrize("batch,K,N,d,D", [(64, 8192, 28672, 10, 24), (2048, 8192, 28672, 10, 24),
                                            (200, 512, 600, 10, 24), (300, 96, 513, 16, 32)])
 def test_workspace_of_tensor_core_path(L, batch, K, N, d, D):
-    """batch >= 64: a 256-byte header, fp16 z [batch][L padded to 64], then batch fp32 scales."""
+    """batch >= 64, lifted GEMM: a 256-byte header, fp16 z [batch][L padded to 64], then batch
+    fp32 scales. Dequantise-once GEMM: the header, fp16 W [N][Kw], fp16 xt [batch][Kw], batch
+    fp32 scales (Kw = ceil(K/d)*d padded to 64)."""
     Lp = -(-lq.lifted_bits(K, d, D) // 64) * 64
-    assert lq.gemm_workspace_bytes(batch, K, N, d, D) == 256 + _r256(batch * Lp * 2 + batch * 4)
+    Kw = -(-(-(-K // d) * d) // 64) * 64
+    for blk in (0, 256):
+        if K % max(blk, 1):
+            continue
+        tc = L.lq_gemm_route_workspace_bytes(batch, K, N, d, D, blk, lq.ROUTE_GEMM_TC)
+        assert tc == 256 + _r256(batch * Lp * 2 + batch * 4)
+        dq = L.lq_gemm_route_workspace_bytes(batch, K, N, d, D, blk, lq.ROUTE_GEMM_DQ)
+        assert dq == 256 + _r256(N * Kw * 2 + batch * Kw * 2 + batch * 4)
+        route = lq.gemm_route(batch, K, N, d, D, blk)
+        assert route in (lq.ROUTE_GEMM_TC, lq.ROUTE_GEMM_DQ)
+        assert lq.gemm_workspace_bytes(batch, K, N, d, D) >= (tc if route == lq.ROUTE_GEMM_TC
+                                                              else dq)
 
 
 def _ptr(v):
@@ -160,3 +177,47 @@ def test_argument_checks_without_gpu(L):
     assert L.lq_device_status(None, ctypes.byref(code), S) == lq.LQ_EINVAL
     for st in range(6):
         assert L.lq_status_string(st)
+
+
+def test_routes_without_gpu(L):
+    """The host-side route query names the kernel family each shape runs on."""
+    assert lq.gemm_route(1, 8192, 28672, 10, 24, 256) == lq.ROUTE_GEMV_I8
+    assert lq.gemm_route(2048, 8192, 28672, 10, 24, 256) == lq.ROUTE_GEMM_DQ
+    assert lq.gemm_route(64, 8192, 28672, 10, 24, 256) == lq.ROUTE_GEMM_TC
+    assert lq.gemm_route(2, 8192, 300, 10, 24, 4096) == lq.ROUTE_GEMV_I8     # block > 256
+    assert lq.gemm_route(8, 4096, 513, 10, 24, 4096) == lq.ROUTE_GEMV_GROUPS
+    assert lq.gemm_route(1, 1048570, 4096, 10, 24, 0) == lq.ROUTE_NONE
+    assert lq.gemm_route(0, 8192, 28672, 10, 24, 256) == -1
+    assert lq.gemm_route(1, 8192, 28672, 10, 24, 3) == -1
+    assert lq.gemm_launches(1, 8192, 28672, 10, 24, 256) == 2
+    assert lq.gemm_launches(1, 1048570, 4096, 10, 24, 0) == 0
+
+
+def test_gemm_rejects_shapes_no_plan_fits_without_gpu(L):
+    fake = ctypes.c_void_p(0x10000)     # never dereferenced: the call is rejected first
+    K, N = 1048570, 4096
+    ws = lq.gemm_workspace_bytes(1, K, N, 10, 24)
+    assert ws > 0
+    rc = L.lq_gemm(fake, lq.LQ_BF16, 1, None, fake, fake, fake, lq.LQ_F16, 10, 24, K, N, fake,
+                   ctypes.c_void_p(0x100000), ws, None)
+    assert rc == lq.LQ_EUNSUPPORTED
+    assert "no GEMV or GEMM plan" in L.lq_last_error().decode()
+
+
+def test_route_workspace_without_gpu(L):
+    """Every route that fits a shape reports its own workspace; a route that does not fit, 0."""
+    args = (2048, 8192, 28672, 10, 24, 256)
+    dq = L.lq_gemm_route_workspace_bytes(*args, lq.ROUTE_GEMM_DQ)
+    tc = L.lq_gemm_route_workspace_bytes(*args, lq.ROUTE_GEMM_TC)
+    assert dq >= 28672 * 8256 * 2 and 0 < tc < dq     # fp16 W is the bulk of the first
+    assert L.lq_gemm_route_workspace_bytes(*args, lq.ROUTE_GEMV_BULK) == 0    # batch > 8
+    assert L.lq_gemm_route_workspace_bytes(*args, lq.ROUTE_NONE) == 0
+    assert L.lq_gemm_route_workspace_bytes(1, 8192, 28672, 10, 24, 256, lq.ROUTE_GEMV_I8) > 0
+    fake = ctypes.c_void_p(0x10000)
+    rc = L.lq_gemm_on_route(fake, lq.LQ_BF16, 1, None, fake, fake, fake, lq.LQ_F16, 10, 24, 8192,
+                            28672, fake, ctypes.c_void_p(0x100000), 1 << 30, 9, None)
+    assert rc == lq.LQ_EINVAL and "route" in L.lq_last_error().decode()
+    rc = L.lq_gemm_on_route(fake, lq.LQ_BF16, 9, None, fake, fake, fake, lq.LQ_F16, 10, 24, 8192,
+                            28672, fake, ctypes.c_void_p(0x100000), 1 << 30, lq.ROUTE_GEMV_BULK,
+                            None)
+    assert rc == lq.LQ_EUNSUPPORTED

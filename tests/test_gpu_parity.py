@@ -99,7 +99,21 @@ SMALL = [
     (1536, 64, 16, 32, 63, 512, synth.BF16, synth.F16),
     (96, 1, 2, 4, 1, 32, synth.F32, synth.F32),
     (4096, 513, 10, 24, 8, 4096, synth.BF16, synth.F16),
+    (8192, 300, 10, 24, 2, 4096, synth.BF16, synth.F16),
+    (4096, 100, 10, 24, 3, 1024, synth.F16, synth.F32),
 ]
+
+
+def test_small_shapes_reach_every_route():
+    """The small shapes run every automatic route; the staged GEMV (chosen only where the
+    two-kernel GEMV cannot take the batch in one launch) and the dequantise-once GEMM are also
+    run on their own routes (test_gemm_small_on_staged_route, test_gpu_gemm_tc.py)."""
+    routes = {lq.gemm_route(b, K, N, d, D, blk) for K, N, d, D, b, blk, _, _ in SMALL}
+    assert routes >= {lq.ROUTE_GEMV_I8, lq.ROUTE_GEMM_TC, lq.ROUTE_GEMV_GROUPS}, routes
+    staged = [s for s in SMALL
+              if lq.lib().lq_gemm_route_workspace_bytes(s[4], s[0], s[1], s[2], s[3], s[5],
+                                                        lq.ROUTE_GEMV_BULK) > 0]
+    assert len(staged) >= 6, staged
 
 
 @pytest.mark.parametrize("K,N,d,D,batch,block,xdt,sdt", SMALL)
@@ -109,7 +123,24 @@ def test_gemm_small_all_rows(orc, K, N, d, D, batch, block, xdt, sdt):
     dl = device_layer(layer)
     y = run_gemm(layer, dl).cpu().numpy()
     ref = oracle_rows(orc, layer, np.arange(N))
-    assert_close(y, ref, f"K={K} N={N} d={d} D={D} batch={batch}")
+    route = lq.gemm_route(batch, K, N, d, D, block)
+    assert_close(y, ref, f"K={K} N={N} d={d} D={D} batch={batch} route={route}")
+
+
+@pytest.mark.parametrize("K,N,d,D,batch,block,xdt,sdt", SMALL)
+def test_gemm_small_on_staged_route(orc, K, N, d, D, batch, block, xdt, sdt):
+    """The staged int8 GEMV (lq_gemm_on_route), all outputs, twice on one workspace."""
+    if lq.lib().lq_gemm_route_workspace_bytes(batch, K, N, d, D, block, lq.ROUTE_GEMV_BULK) == 0:
+        pytest.skip("the staged GEMV's plan does not fit this shape")
+    layer = synth.make_layer("small", 99, K + N, K, N, d, D, batch, block=block, x_dtype=xdt,
+                             s_dtype=sdt)
+    dl = device_layer(layer)
+    ws = lq.new_workspace(batch, K, N, d, D, block=block, route=lq.ROUTE_GEMV_BULK)
+    ref = oracle_rows(orc, layer, np.arange(N))
+    for _ in range(2):
+        y = run_gemm(layer, dl, ws, route=lq.ROUTE_GEMV_BULK).cpu().numpy()
+        assert_close(y, ref, f"staged K={K} N={N} d={d} D={D} batch={batch}")
+    assert lq.device_status(ws) == (lq.LQ_OK, 0)
 
 
 def test_gemm_identity_special_case(orc):
@@ -150,7 +181,10 @@ def _sample_rows(N, n, seed):
     return np.unique(np.concatenate([r, [0, N - 1]]))
 
 
-def _check_workload(orc, cfg, max_rows=96, max_tokens=48):
+def _check_workload(orc, cfg, max_rows=None, max_tokens=48):
+    """Every output of every layer of a workload against the oracle, except on the 2048-token
+    prefill, where the oracle's cost calls for a sample of rows and tokens (max_rows x
+    max_tokens, chosen by a seeded draw plus the first and last row)."""
     specs = synth.workload_specs(cfg)
     cache = {}
     for spec in specs:
@@ -164,13 +198,14 @@ def _check_workload(orc, cfg, max_rows=96, max_tokens=48):
         dl = dict(cache[key])
         dl["x"] = to_torch_x(layer).cuda()
         y = run_gemm(layer, dl).cpu().numpy()
-        rows = np.arange(N) if N <= max_rows else _sample_rows(N, max_rows, cfg * 7 + li)
+        rows = np.arange(N) if max_rows is None or N <= max_rows else \
+            _sample_rows(N, max_rows, cfg * 7 + li)
         toks = None if batch <= max_tokens else np.sort(_rng(cfg).choice(batch, max_tokens,
                                                                           replace=False))
         ref = oracle_rows(orc, layer, rows, toks)
         got = y[:, rows] if toks is None else y[toks][:, rows]
         rel, mx = assert_close(got, ref, name)
-        print(f"{name}: rel_l2={rel:.2e} max_abs/rms={mx:.2e}")
+        print(f"{name}: {got.size} outputs, rel_l2={rel:.2e} max_abs/rms={mx:.2e}")
     cache.clear()
     torch.cuda.empty_cache()
 
@@ -192,4 +227,4 @@ def test_workload_bitwidth_sweep(orc):
 
 
 def test_workload_prefill(orc):
-    _check_workload(orc, 5)
+    _check_workload(orc, 5, max_rows=512)

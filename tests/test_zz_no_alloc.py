@@ -3,8 +3,8 @@
 Such callers (a plugin or serving backend whose device memory belongs to a host framework, or
 code that runs where allocating is not allowed) cannot pass lq_gemm a workspace; this entry
 point keeps its scratch in a fixed device array owned by the library. The test calls it through
-the C ABI and compares it with lq_gemm on the same inputs, twice in a row (the second call finds
-the scratch as the first call left it). It runs last so that a failure here does not hide the
+the C ABI and compares it with the fp64 oracle, and with lq_gemm on the same inputs, twice in a
+row (the second call finds the scratch as the first call left it). It runs last so that a failure here does not hide the
 other GPU tests, and passes both on its own and after them.
 """
 import ctypes
@@ -15,7 +15,7 @@ import torch
 
 import fractional_bit_weight_b200 as lq
 from fractional_bit_weight_b200 import synth
-from gpu_helpers import assert_close, device_layer
+from gpu_helpers import assert_close, device_layer, oracle_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -32,16 +32,20 @@ def _call_noalloc(layer, dl, y):
 
 @pytest.mark.parametrize("K,N,d,D,batch", [(4096, 4096, 10, 24, 1), (8192, 3000, 3, 8, 3),
                                            (28672, 1024, 10, 24, 2), (256, 128, 2, 5, 1)])
-def test_noalloc_matches_gemm_twice(K, N, d, D, batch):
+def test_noalloc_matches_oracle_and_gemm_twice(orc, K, N, d, D, batch):
     layer = synth.make_layer("noalloc", 11, K + N + batch, K, N, d, D, batch)
     dl = device_layer(layer)
-    ref = lq.gemm(dl["x"], dl["packed"], dl["M"], dl["s"], d, D, sign=dl["sign"],
-                  block=layer.block).cpu().numpy()
+    ref = oracle_rows(orc, layer, np.arange(N))
+    y_gemm = lq.gemm(dl["x"], dl["packed"], dl["M"], dl["s"], d, D, sign=dl["sign"],
+                     block=layer.block).cpu().numpy()
+    what = f"K={K} N={N} d={d} D={D} batch={batch}"
     for _ in range(2):
         y = torch.full((batch, N), float("nan"), dtype=torch.float32, device="cuda")
         assert _call_noalloc(layer, dl, y) == lq.LQ_OK, lq.lib().lq_last_error().decode()
         torch.cuda.synchronize()
-        assert_close(y.cpu().numpy(), ref, f"noalloc K={K} N={N} d={d} D={D} batch={batch}")
+        got = y.cpu().numpy()
+        assert_close(got, ref, f"noalloc vs oracle, {what}")
+        assert_close(got, y_gemm, f"noalloc vs lq_gemm, {what}")
 
 
 def test_noalloc_rejects_what_does_not_fit():
