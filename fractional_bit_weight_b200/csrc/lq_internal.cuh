@@ -116,11 +116,15 @@ struct BsPlan {
   int R;              // row ranges
   int rq, rrem;       // rows per range: rq + (range < rrem)
   int rows_max;       // rq + 1
+  int rows_per_stage;  // 16 or 32
   int wch;            // chunks per stage window
   int stride;         // shared-memory row stride of a stage
+  int whole;          // 1: a stage is one copy of whole contiguous rows
+  uint32_t perm;      // MMA row -> stage row inside each group of 8 (nibbles)
   int NS;             // ring stages
+  int early_stages;   // stages issued before the operand is built
   int nctas;          // S * R
-  int xs_floats;      // whitened inputs of a slice, per token
+  int xs_floats;      // staged, whitened inputs of the slice, per token
   size_t smem;        // dynamic shared memory per CTA
   size_t frag_smem;   // shared memory: the slice's fragments
   size_t prep_smem;   // shared memory: whitening, z and M scratch
