@@ -73,11 +73,11 @@ struct WsLayout {
   int path;          // LQ_ROUTE_*: 0 int8 tensor-core GEMV (batch <= 8, two kernels); 1 no plan
                      // fits; 2 tcgen05 GEMM (batch >= lq::kTcMinBatch); 3 the int8 GEMV once
                      // per group of gs tokens (when no single-launch plan fits); 4 the
-                     // staged int8 GEMV (batch <= 8, one kernel); 5 the
+                     // staged int8 GEMV (batch <= 8, prep + TMA-staged GEMV); 5 the
                      // dequantise-once GEMM (fp16 W, dense tcgen05 GEMM)
   size_t counters;   // uint32 completion counters of the split-K reduction
   size_t z;          // paths 0/3: prep output (fragments, weights, sums); 2: fp16 z and token
-                     // scales; 4: fragments, token scales, chunk sums
+                     // scales; 4: prep output (fragments, chunk sums, token scales)
   size_t partials;   // float [slices][batch][N]
   size_t total;
   lq::G8Plan g8;
@@ -124,8 +124,14 @@ WsLayout layout_gemm(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D, 
     if (tc_s < gemv_s) w.path = 2;
   }
   if (w.path == 1 && w.tc.ok && batch > 8) w.path = 2;
-  // the staged GEMV serves batches the two-kernel GEMV cannot take in one launch
+  // the staged GEMV serves batches the register-streamed GEMV cannot take in one launch, and
+  // one or two tokens on layers of >= 32 MB of codes, where its TMA stream measured faster on
+  // B200 (Llama-3-70B MLP shapes: 29.9 against 31.5 us at one token); on smaller layers and at
+  // 3..8 tokens the register-streamed GEMV measured faster
   if (w.bs.ok && w.path != 0) w.path = 4;
+  if (w.bs.ok && w.path == 0 && batch <= 2 &&
+      (double)N * (double)row_stride_bytes(K, d, D) >= 32.0 * 1024 * 1024)
+    w.path = 4;
   // the tensor-core routes: the lifted GEMM contracts over L coordinates; the dequantise-once
   // GEMM over G*d inputs (D/d times fewer MMA flops) after writing and reading fp16 W once.
   // Rough B200 costs: ~1.0 PFLOP/s lifted, ~1.3 PFLOP/s dense, ~5 TB/s for W's two passes.
@@ -145,7 +151,7 @@ WsLayout layout_gemm(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D, 
     nz = (w.dq.w_bytes + w.dq.x_bytes + w.dq.scale_bytes + 3) / 4;
   } else if (w.path == 4) {
     ncounters = (size_t)w.bs.R;
-    nz = (w.bs.sumz_bytes + 3) / 4;   // per-slice sums of z
+    nz = (w.bs.frag_bytes + w.bs.csum_bytes + w.bs.stok_bytes + 3) / 4;   // prep output
     npartials = w.bs.gacc_bytes / 4;  // int32 totals
   } else if (w.path == 3) {
     // the groups run one after the other on the stream and share the scratch
@@ -317,7 +323,7 @@ int32_t lq_gemm_launches(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t
   const WsLayout lay = layout_gemm(batch, K, N, d, D, block);
   // path 4: one kernel; paths 0 and 2: a prologue kernel and a contraction kernel, per token
   // group on path 3; path 1: nothing (the call is rejected)
-  if (lay.path == 4) return 1;
+  if (lay.path == 4) return 2;
   if (lay.path == 1) return 0;
   if (lay.path == 5) return 3;   // W, xt, GEMM
   return lay.path == 3 ? 2 * ((batch + lay.gs - 1) / lay.gs) : 2;
@@ -364,7 +370,9 @@ lq_status gemm_impl(const void* x, lq_dtype xdt, int32_t batch, const lq_whiten_
   float* partials = reinterpret_cast<float*>(ws + lay.partials);
   if (lay.path == 4) {
     lq::BsScratch sc{};
-    sc.sumz = reinterpret_cast<float*>(ws + lay.z);
+    sc.frags = reinterpret_cast<uint8_t*>(ws + lay.z);
+    sc.csum = reinterpret_cast<float*>(ws + lay.z + lay.bs.frag_bytes);
+    sc.stok = reinterpret_cast<float*>(ws + lay.z + lay.bs.frag_bytes + lay.bs.csum_bytes);
     sc.gacc = reinterpret_cast<int*>(ws + lay.partials);
     sc.counters = counters;
     sc.status = reinterpret_cast<uint32_t*>(ws);

@@ -105,8 +105,9 @@ cudaError_t launch_gemm_tc(const TcPlan& pl, const void* x, int xdt, int32_t bat
                            const uint32_t* packed, int64_t row_bytes, int32_t N, const void* s,
                            int sdt, float* y, void* scratch, uint32_t* status, cudaStream_t st);
 
-// Plan of the staged int8 tensor-core GEMV (batch <= 8): one launch of S K-slices x R row
-// ranges, one CTA per SM; each CTA builds its slice's activation operand itself.
+// Plan of the staged int8 tensor-core GEMV (batch <= 8): a prep kernel, one CTA per 512-bit
+// chunk, writes the activation fragments; the GEMV (S K-slices x R row ranges, one CTA per SM,
+// programmatic dependent launch) streams the codes through shared memory with TMA.
 struct BsPlan {
   bool ok;
   int nt;             // 8-column MMA tiles (2 tokens each)
@@ -117,26 +118,28 @@ struct BsPlan {
   int rq, rrem;       // rows per range: rq + (range < rrem)
   int rows_max;       // rq + 1
   int rows_per_stage;  // 16 or 32
-  int wch;            // chunks per stage window
-  int stride;         // shared-memory row stride of a stage
-  int whole;          // 1: a stage is one copy of whole contiguous rows
-  uint32_t perm;      // MMA row -> stage row inside each group of 8 (nibbles)
+  int wch;            // chunks per stage window (odd)
+  int stride;         // shared-memory row stride of a stage (64 * wch)
   int NS;             // ring stages
-  int early_stages;   // stages issued before the operand is built
   int nctas;          // S * R
-  int xs_floats;      // staged, whitened inputs of the slice, per token
-  size_t smem;        // dynamic shared memory per CTA
-  size_t frag_smem;   // shared memory: the slice's fragments
-  size_t prep_smem;   // shared memory: whitening, z and M scratch
-  size_t sumz_bytes;  // scratch: per-slice sums of z [S][batch] (S > 1)
+  int xs_floats;      // prep: whitened inputs of one chunk, per token
+  size_t smem;        // GEMV dynamic shared memory per CTA
+  size_t frag_smem;   // GEMV shared memory: the slice's fragments and a zero block
+  size_t prep_smem;   // prep dynamic shared memory per CTA
+  size_t frag_bytes;  // scratch: fragments [batch][nchunk][1536]
+  size_t csum_bytes;  // scratch: per-chunk sums of z [nchunk][batch]
+  size_t stok_bytes;  // scratch: per-token scales [batch]
   size_t gacc_bytes;  // scratch: int32 totals [batch][N][4] (S > 1), zero at rest
 };
 BsPlan plan_gemv_bs(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, int32_t D,
                     int32_t Bh);
-// Global scratch of one call (used when S > 1): gacc and counters [R] must be zero before the
-// first call and are left zero by every call; sumz is rewritten by every call.
+// Global scratch of one call: frags, csum and stok are rewritten by every call (16-byte
+// aligned); gacc and counters [R] (used when S > 1) must be zero before the first call and are
+// left zero by every call.
 struct BsScratch {
-  float* sumz;
+  uint8_t* frags;
+  float* csum;
+  float* stok;
   int* gacc;
   uint32_t* counters;
   uint32_t* status;

@@ -156,8 +156,8 @@ LQ_API int32_t lq_gemm_launches(int32_t batch, int32_t K, int32_t N, int32_t d, 
  *   LQ_ROUTE_NONE        no plan fits the shape: lq_gemm returns LQ_EUNSUPPORTED
  *   LQ_ROUTE_GEMM_TC     tcgen05 tensor-core GEMM over fp16 z (batch >= 64, or where cheaper)
  *   LQ_ROUTE_GEMV_GROUPS LQ_ROUTE_GEMV_I8 once per group of tokens
- *   LQ_ROUTE_GEMV_BULK   int8 tensor-core GEMV with bulk-copied code rows, one cooperative
- *                        kernel (batch <= 8 where its plan fits)
+ *   LQ_ROUTE_GEMV_BULK   int8 tensor-core GEMV, prologue + contraction kernels, the codes
+ *                        streamed through shared memory by TMA (batch <= 8 where its plan fits)
  *   LQ_ROUTE_GEMM_DQ     W = blockwise M b dequantised once to fp16 in the workspace, then a
  *                        dense tcgen05 GEMM of fp16 T(x) against W (large batches, where its
  *                        D/d-times smaller contraction outweighs writing and reading W) */

@@ -102,12 +102,12 @@ def test_gemm_launches(L):
                                             (28672, 8192, 4), (256, 128, 8), (40, 64, 8)])
 def test_small_batches_run_as_one_gemv(L, K, N, max_single):
     """Up to 4 tokens on the Llama-3-70B MLP shapes, up to 8 on 4096- and 8192-wide layers, the
-    batch runs as one int8 GEMV (one bulk-staged kernel, or prep + contraction) instead of
+    batch runs as one int8 GEMV (prep + contraction: register-streamed or TMA-staged) instead of
     token groups."""
     for b in range(1, max_single + 1):
         route = lq.gemm_route(b, K, N, 10, 24, 256)
         assert route in (lq.ROUTE_GEMV_BULK, lq.ROUTE_GEMV_I8), (b, route)
-        assert lq.gemm_launches(b, K, N, 10, 24, 256) == (1 if route == lq.ROUTE_GEMV_BULK else 2)
+        assert lq.gemm_launches(b, K, N, 10, 24, 256) == 2
 
 
 @pytest.mark.parametrize("batch,K,N,d,D", [(64, 8192, 28672, 10, 24), (2048, 8192, 28672, 10, 24),
@@ -181,7 +181,12 @@ def test_argument_checks_without_gpu(L):
 
 def test_routes_without_gpu(L):
     """The host-side route query names the kernel family each shape runs on."""
-    assert lq.gemm_route(1, 8192, 28672, 10, 24, 256) == lq.ROUTE_GEMV_I8
+    # one or two tokens on a layer of >= 32 MB of codes: the TMA-staged GEMV; else the
+    # register-streamed one up to 8 tokens
+    assert lq.gemm_route(1, 8192, 28672, 10, 24, 256) == lq.ROUTE_GEMV_BULK
+    assert lq.gemm_route(2, 28672, 8192, 10, 24, 256) == lq.ROUTE_GEMV_BULK
+    assert lq.gemm_route(3, 8192, 28672, 10, 24, 256) == lq.ROUTE_GEMV_I8
+    assert lq.gemm_route(1, 4096, 4096, 10, 24, 256) == lq.ROUTE_GEMV_I8
     assert lq.gemm_route(2048, 8192, 28672, 10, 24, 256) == lq.ROUTE_GEMM_DQ
     assert lq.gemm_route(64, 8192, 28672, 10, 24, 256) == lq.ROUTE_GEMM_TC
     assert lq.gemm_route(2, 8192, 300, 10, 24, 4096) == lq.ROUTE_GEMV_I8     # block > 256
