@@ -40,14 +40,32 @@ struct Params {
   float* err;        // [N][G] or nullptr
 };
 
-// Shared tables, zero beyond d rows / columns so that loops may run to the template size.
-struct Tables {
+// Shared tables, zero beyond d rows / columns so that loops may run to the template size. The
+// walks read one column per step, the same for every lane of a warp: the column-major copies
+// CM and CP serve those reads as 16-byte broadcast loads.
+struct __align__(16) Tables {
+  float CM[32][kMaxd];      // CM[j][i] = M[i][j]
+  float CP[32][kMaxd];      // CP[k][i] = P[i][k] (seeded)
   float M[kMaxd][32];       // M, [i][j]
   float Minv[kMaxd][kMaxd]; // M_S^-1 (seeded)
   float P[kMaxd][32];       // M_S^-1 M_F, [i][k] (seeded)
   float A[kMaxd][2 * kMaxd];// Gauss-Jordan scratch
   int singular;
 };
+
+// column j of a column-major table (kMaxd floats, 16-byte aligned) into registers
+template <int DM>
+__device__ __forceinline__ void load_column(const float* col, float (&v)[DM]) {
+  const float4* c4 = reinterpret_cast<const float4*>(col);
+#pragma unroll
+  for (int q = 0; q < (DM + 3) / 4; ++q) {
+    const float4 a = c4[q];
+    if (4 * q + 0 < DM) v[4 * q + 0] = a.x;
+    if (4 * q + 1 < DM) v[4 * q + 1] = a.y;
+    if (4 * q + 2 < DM) v[4 * q + 2] = a.z;
+    if (4 * q + 3 < DM) v[4 * q + 3] = a.w;
+  }
+}
 
 // M_S^-1 by Gauss-Jordan with partial pivoting (one thread; d <= 16), then P = M_S^-1 M_F.
 __device__ void build_tables(const Params& p, Tables& t) {
@@ -101,6 +119,12 @@ __device__ void build_tables(const Params& p, Tables& t) {
     t.P[i][k] = a;
   }
   __syncthreads();
+  for (int e = tid; e < 32 * kMaxd; e += blockDim.x) {
+    const int j = e / kMaxd, i = e - j * kMaxd;
+    t.CM[j][i] = t.M[i][j];
+    t.CP[j][i] = t.P[i][j];
+  }
+  __syncthreads();
 }
 
 __device__ __forceinline__ void warp_argmin(float& dist, uint32_t& idx) {
@@ -148,8 +172,10 @@ __device__ void search_exact(const Params& p, const Tables& t, const float (&w)[
     if (s + 1 < cnt) {                              // flip coordinate ctz(s+1): b_j -> -b_j
       const int j = __ffs(s + 1) - 1;
       const float sg2 = ((code >> j) & 1) ? -2.f : 2.f;
+      float cj[DM];
+      load_column<DM>(t.CM[j], cj);
 #pragma unroll
-      for (int i = 0; i < DM; ++i) r[i] = fmaf(sg2, t.M[i][j], r[i]);
+      for (int i = 0; i < DM; ++i) r[i] = fmaf(sg2, cj[i], r[i]);
       code ^= 1u << j;
     }
   }
@@ -166,7 +192,7 @@ __device__ void search_seeded(const Params& p, const Tables& t, const float (&w)
   best_f = 0xffffffffu;
   best_mask = 0;
   if (F < 5 && lane >= (1 << F)) return;
-  float rF[DM], u[DM], e[DM];
+  float u[DM], e[DM];
   uint32_t f = (uint32_t)lane << lg, mask = 0;      // mask bit i: b_i = -1 (i < d)
   for (uint32_t s = 0; s < cnt; ++s) {
     if ((s & (kRefresh - 1)) == 0) {
@@ -174,6 +200,7 @@ __device__ void search_seeded(const Params& p, const Tables& t, const float (&w)
       // all of M_S^-1 and M_S in registers across the walk for this rare step
       const volatile float* Mv = &t.M[0][0];
       const volatile float* Iv = &t.Minv[0][0];
+      float rF[DM];
 #pragma unroll
       for (int i = 0; i < DM; ++i) {
         float a = w[i];
@@ -209,12 +236,14 @@ __device__ void search_seeded(const Params& p, const Tables& t, const float (&w)
     if (s + 1 < cnt) {                              // flip free coordinate k = ctz(s+1)
       const int k = __ffs(s + 1) - 1;
       const float sg2 = ((f >> k) & 1) ? -2.f : 2.f;  // r_F moves by sg2 * M[:, d+k]
+      float mk[DM], pk[DM];
+      load_column<DM>(t.CM[d + k], mk);
+      load_column<DM>(t.CP[k], pk);
+      // e moves with r_F, u by the column of P
 #pragma unroll
       for (int i = 0; i < DM; ++i) {
-        const float dr = sg2 * t.M[i][d + k];
-        rF[i] += dr;
-        e[i] += dr;
-        u[i] = fmaf(sg2, t.P[i][k], u[i]);
+        e[i] = fmaf(sg2, mk[i], e[i]);
+        u[i] = fmaf(sg2, pk[i], u[i]);
       }
       f ^= 1u << k;
       uint32_t nmask = 0;
@@ -225,8 +254,10 @@ __device__ void search_seeded(const Params& p, const Tables& t, const float (&w)
       for (uint32_t fl = nmask ^ mask; fl; fl &= fl - 1) {
         const int c = __ffs(fl) - 1;
         const float g2 = ((mask >> c) & 1) ? -2.f : 2.f;
+        float mc[DM];
+        load_column<DM>(t.CM[c], mc);
 #pragma unroll
-        for (int i = 0; i < DM; ++i) e[i] = fmaf(g2, t.M[i][c], e[i]);
+        for (int i = 0; i < DM; ++i) e[i] = fmaf(g2, mc[i], e[i]);
       }
       mask = nmask;
     }
@@ -234,7 +265,7 @@ __device__ void search_seeded(const Params& p, const Tables& t, const float (&w)
 }
 
 template <int DM, bool kSeeded>
-__global__ void __launch_bounds__(kThreads) encode_kernel(const Params p) {
+__global__ void __launch_bounds__(kThreads, 4) encode_kernel(const Params p) {
   __shared__ Tables t;
   build_tables(p, t);
   const int lane = threadIdx.x & 31;
