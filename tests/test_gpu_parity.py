@@ -105,9 +105,10 @@ SMALL = [
 
 
 def test_small_shapes_reach_every_route():
-    """The small shapes run every automatic route; the staged GEMV (chosen only where the
-    two-kernel GEMV cannot take the batch in one launch) and the dequantise-once GEMM are also
-    run on their own routes (test_gemm_small_on_staged_route, test_gpu_gemm_tc.py)."""
+    """The small shapes run every automatic route; the staged GEMV (chosen for one or two
+    tokens on layers of >= 32 MB of codes, and where the register-streamed GEMV cannot take the
+    batch in one launch) and the dequantise-once GEMM are also run on their own routes
+    (test_gemm_small_on_staged_route, test_gpu_gemm_tc.py)."""
     routes = {lq.gemm_route(b, K, N, d, D, blk) for K, N, d, D, b, blk, _, _ in SMALL}
     assert routes >= {lq.ROUTE_GEMV_I8, lq.ROUTE_GEMM_TC, lq.ROUTE_GEMV_GROUPS}, routes
     staged = [s for s in SMALL
@@ -141,6 +142,19 @@ def test_gemm_small_on_staged_route(orc, K, N, d, D, batch, block, xdt, sdt):
         y = run_gemm(layer, dl, ws, route=lq.ROUTE_GEMV_BULK).cpu().numpy()
         assert_close(y, ref, f"staged K={K} N={N} d={d} D={D} batch={batch}")
     assert lq.device_status(ws) == (lq.LQ_OK, 0)
+
+
+def test_staged_route_two_tokens_full_size(orc):
+    """Two tokens on the Llama-3-70B gate/up shape (8192 -> 28672, d=10, D=24, block 256, bf16
+    x, f16 s) take the staged GEMV by default: all 28672 x 2 outputs against the oracle."""
+    K, N, d, D, batch = 8192, 28672, 10, 24, 2
+    assert lq.gemm_route(batch, K, N, d, D, 256) == lq.ROUTE_GEMV_BULK
+    layer = synth.make_layer("gateup2", 12, 0, K, N, d, D, batch, block=256, x_dtype=synth.BF16,
+                             s_dtype=synth.F16)
+    dl = device_layer(layer)
+    y = run_gemm(layer, dl).cpu().numpy()
+    ref = oracle_rows(orc, layer, np.arange(N))
+    assert_close(y, ref, "staged GEMV, 2 tokens, 8192 x 28672")
 
 
 def test_gemm_identity_special_case(orc):
