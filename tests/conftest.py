@@ -20,3 +20,15 @@ def pytest_configure(config):
 def orc():
     import oracle
     return oracle
+
+
+def pytest_terminal_summary(terminalreporter):
+    """The largest errors the parity comparisons observed, by what was compared."""
+    helpers = sys.modules.get("gpu_helpers")
+    if helpers is None or not getattr(helpers, "OBSERVED", None):
+        return
+    rows = sorted(helpers.OBSERVED, key=lambda r: -r[1])
+    terminalreporter.section("observed parity errors (largest relative L2 first)")
+    for what, rel, mx in rows[:40]:
+        terminalreporter.write_line(f"rel-L2 {rel:.2e}  max-abs/RMS {mx:.2e}  {what}")
+    terminalreporter.write_line(f"{len(rows)} comparisons")

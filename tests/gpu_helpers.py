@@ -68,8 +68,14 @@ def errors(y, ref):
     return rel, mx
 
 
+# every comparison made by assert_close in this session: (what, rel-L2, max-abs/RMS), printed in
+# the terminal summary (tests/conftest.py)
+OBSERVED = []
+
+
 def assert_close(y, ref, what=""):
     rel, mx = errors(y, ref)
+    OBSERVED.append((what, rel, mx))
     assert np.isfinite(y).all(), what
     assert rel <= REL_L2, f"{what}: relative L2 error {rel:.3e} > {REL_L2}"
     assert mx <= MAX_ABS_OVER_RMS, f"{what}: max-abs/RMS {mx:.3e} > {MAX_ABS_OVER_RMS}"

@@ -218,7 +218,8 @@ def _check_workload(orc, cfg, max_rows=None, max_tokens=48):
                                                                           replace=False))
         ref = oracle_rows(orc, layer, rows, toks)
         got = y[:, rows] if toks is None else y[toks][:, rows]
-        rel, mx = assert_close(got, ref, name)
+        route = lq.gemm_route(batch, K, N, d, D, layer.block)
+        rel, mx = assert_close(got, ref, f"{name} route={route}")
         print(f"{name}: {got.size} outputs, rel_l2={rel:.2e} max_abs/rms={mx:.2e}")
     cache.clear()
     torch.cuda.empty_cache()
