@@ -128,6 +128,11 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// shared-memory integer add without a returned value
+__device__ __forceinline__ void red_add_shared(int* p, int v) {
+  asm volatile("red.shared.add.s32 [%0], %1;" ::"r"(sm100::smem_u32(p)), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -597,9 +602,8 @@ __global__ void __launch_bounds__(bs::kThreads, 1)
             for (int c = 0; c < CH; ++c) v += acc[nt][h][c][r];
             const int rr = rbase + 16 * h + g + 8 * (r >> 1);
             const int col = 2 * t + (r & 1);           // column within the tile
-            const int tok = 2 * nt + (col >> 2), pl = col & 3;
-            if (rr < rows && pl < bs::kPlanes && tok < P.batch && v != 0)
-              atomicAdd(&rowacc[rr * 8 * NT + 8 * nt + col], v);
+            const bool live = rr < rows && (col & 3) < bs::kPlanes && 2 * nt + (col >> 2) < P.batch;
+            red_add_shared(&rowacc[min(rr, rows - 1) * 8 * NT + 8 * nt + col], live ? v : 0);
 #pragma unroll
             for (int c = 0; c < CH; ++c) acc[nt][h][c][r] = 0;
           }
@@ -716,7 +720,7 @@ BsPlan plan_gemv_bs(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, i
   if (p.prep_smem > 200 * 1024) return p;
   const int sms = bs_sm_count();
   constexpr size_t kBudget = 224 * 1024;
-  for (int S = 1; S <= 16; ++S) {
+  for (int S = 1; S <= 16 && !p.ok; ++S) {
     const int sc = (p.nchunk + S - 1) / S;
     if (S > 1 && (p.nchunk + sc - 1) / sc != S) continue;   // no empty slice
     const int R = std::max(1, std::min(sms / S, (N + 15) / 16));

@@ -25,7 +25,13 @@ def orc():
 def pytest_terminal_summary(terminalreporter):
     """The largest errors the parity comparisons observed, by what was compared."""
     helpers = sys.modules.get("gpu_helpers")
-    if helpers is None or not getattr(helpers, "OBSERVED", None):
+    if helpers is None:
+        return
+    if getattr(helpers, "NOTES", None):
+        terminalreporter.section("figures reported by the tests")
+        for line in helpers.NOTES:
+            terminalreporter.write_line(line)
+    if not getattr(helpers, "OBSERVED", None):
         return
     rows = sorted(helpers.OBSERVED, key=lambda r: -r[1])
     terminalreporter.section("observed parity errors (largest relative L2 first)")

@@ -71,6 +71,8 @@ def errors(y, ref):
 # every comparison made by assert_close in this session: (what, rel-L2, max-abs/RMS), printed in
 # the terminal summary (tests/conftest.py)
 OBSERVED = []
+# other figures a test reports (one line each), printed in the same summary
+NOTES = []
 
 
 def assert_close(y, ref, what=""):
