@@ -399,12 +399,12 @@ __global__ void __launch_bounds__(bs::kPrepThreads) gemv_bs_prep_kernel(const Bs
   }
 }
 
-// One item: HT tiles of 16 rows x one 64-byte chunk (UP: the tiles past the first hold rows),
-// NT tiles of B (8 columns each), CH accumulator chains per (tile, B tile).
-template <int NT, int HT, int CH, bool UP>
+// One item: the first HA of HT tiles of 16 rows (those that hold rows) x one 64-byte chunk, NT
+// tiles of B (8 columns each), CH accumulator chains per (tile, B tile).
+template <int NT, int HT, int CH, int HA>
 __device__ __forceinline__ void run_item(uint32_t arow, int stride, uint32_t fb, const uint32_t (&fofs)[NT],
                                          uint32_t mstep, int (&acc)[NT][HT][CH][4]) {
-  constexpr int HA = UP ? HT : 1;   // tiles with rows
+  static_assert(HA >= 1 && HA <= HT, "tiles with rows");
   uint4 u[HA][2];
 #pragma unroll
   for (int h = 0; h < HA; ++h) {
@@ -433,6 +433,20 @@ __device__ __forceinline__ void run_item(uint32_t arow, int stride, uint32_t fb,
         }
       }
     }
+  }
+}
+
+// This warp's items of one stage: chunks first, first + 16, ... of the window.
+template <int NT, int HT, int CH, int HA>
+__device__ __forceinline__ void run_window(int first, int nitems, uint32_t fwin, uint32_t sbase, int stride,
+                                           const uint32_t (&fofs)[NT], uint32_t zero_u32, uint32_t mstep,
+                                           int (&acc)[NT][HT][CH][4]) {
+  for (int cw = first; cw < nitems; cw += bs::kWarps) {
+    const uint32_t fb = fwin + (uint32_t)cw * bs::kTokBytes;
+    uint32_t fo[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) fo[nt] = fofs[nt] == 0xffffffffu ? zero_u32 - fb : fofs[nt];
+    run_item<NT, HT, CH, HA>(sbase + 64 * cw, stride, fb, fo, mstep, acc);
   }
 }
 
@@ -568,22 +582,12 @@ __global__ void __launch_bounds__(bs::kThreads, 1)
     }
     const uint32_t sbase = ring_u32 + (uint32_t)(k * stage_bytes) + (uint32_t)(g * stride + 16 * t);
     const uint32_t fwin = frag_u32 + (uint32_t)(win * P.wch) * bs::kTokBytes;
-    if (HT == 1 || nr > 16) {
-      for (int cw = first; cw < nitems; cw += bs::kWarps) {
-        const uint32_t fb = fwin + (uint32_t)cw * bs::kTokBytes;
-        uint32_t fo[NT];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) fo[nt] = fofs[nt] == 0xffffffffu ? zero_u32 - fb : fofs[nt];
-        run_item<NT, HT, CH, true>(sbase + 64 * cw, stride, fb, fo, mstep, acc);
-      }
+    // the stage's tiles of 16 rows that hold rows of the range
+    const int live = (nr + 15) >> 4;
+    if (live >= HT) {
+      run_window<NT, HT, CH, HT>(first, nitems, fwin, sbase, stride, fofs, zero_u32, mstep, acc);
     } else {
-      for (int cw = first; cw < nitems; cw += bs::kWarps) {
-        const uint32_t fb = fwin + (uint32_t)cw * bs::kTokBytes;
-        uint32_t fo[NT];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) fo[nt] = fofs[nt] == 0xffffffffu ? zero_u32 - fb : fofs[nt];
-        run_item<NT, HT, CH, false>(sbase + 64 * cw, stride, fb, fo, mstep, acc);
-      }
+      run_window<NT, HT, CH, 1>(first, nitems, fwin, sbase, stride, fofs, zero_u32, mstep, acc);
     }
     first = (first - nitems) & (bs::kWarps - 1);
     __syncwarp();
