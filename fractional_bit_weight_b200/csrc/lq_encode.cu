@@ -16,7 +16,8 @@
 // one coordinate flips per step and the residual r = w - M b (exact) or r_F = w - M_F b_F,
 // u = M_S^-1 r_F and e = r_F - M_S b_S (seeded) change by one column each, d operations per
 // step instead of d^2: u moves by a column of P = M_S^-1 M_F, e by the same column of M_F plus
-// one column of M_S for every solved sign that flips. Every 256 steps the lane recomputes its
+// one column of M_S for every solved sign that flips. For d <= 10 the seeded walk instead reads
+// e = r_F - T[b_S] from a shared-memory table of M_S b_S over all 2^d solved sign patterns. Every 256 steps the lane recomputes its
 // state from the definition, which bounds fp32 drift. The warp then takes the minimum of
 // (distance, index) over its lanes. Arithmetic is fp32; where two candidates lie within fp32
 // rounding of each other the pick may differ from an fp64 search, never its distance by more
@@ -264,10 +265,90 @@ __device__ void search_seeded(const Params& p, const Tables& t, const float (&w)
   }
 }
 
-template <int DM, bool kSeeded>
+// Seeded search with a table of M_S b_S over all 2^d solved sign patterns (d <= 10): the walk
+// keeps r_F and u, and e = r_F - T[mask] is read per step instead of being moved by one column
+// of M_S per solved sign that flips. T: [2^d][DP] floats, DP = DM rounded up to 4.
+template <int DM>
+__device__ void search_seeded_table(const Params& p, const Tables& t, const float* __restrict__ T,
+                                    const float (&w)[DM], int lane, float& best_dist,
+                                    uint32_t& best_f, uint32_t& best_mask) {
+  constexpr int DP = (DM + 3) / 4 * 4;
+  const int d = p.d, F = p.D - p.d;
+  const int lg = F >= 5 ? F - 5 : 0;
+  const uint32_t cnt = 1u << lg;
+  best_dist = INFINITY;
+  best_f = 0xffffffffu;
+  best_mask = 0;
+  if (F < 5 && lane >= (1 << F)) return;
+  float rF[DM], u[DM];
+  uint32_t f = (uint32_t)lane << lg, mask = 0;      // mask bit i: b_i = -1 (i < d)
+  for (uint32_t s = 0; s < cnt; ++s) {
+    if ((s & (kRefresh - 1)) == 0) {
+      const volatile float* Mv = &t.M[0][0];
+      const volatile float* Iv = &t.Minv[0][0];
+#pragma unroll
+      for (int i = 0; i < DM; ++i) {
+        float a = w[i];
+        for (int k = 0; k < F; ++k) a -= Mv[i * 32 + d + k] * (((f >> k) & 1) ? -1.f : 1.f);
+        rF[i] = a;
+      }
+      mask = 0;
+#pragma unroll
+      for (int i = 0; i < DM; ++i) {
+        float a = 0.f;
+#pragma unroll
+        for (int c = 0; c < DM; ++c) a = fmaf(Iv[i * kMaxd + c], rF[c], a);
+        u[i] = a;
+        if (i < d && a < 0.f) mask |= 1u << i;
+      }
+    }
+    float tm[DM];
+    load_column<DM>(T + (size_t)mask * DP, tm);
+    float dist = 0.f;
+#pragma unroll
+    for (int i = 0; i < DM; ++i) {
+      const float e = rF[i] - tm[i];
+      dist = fmaf(e, e, dist);
+    }
+    if (dist < best_dist || (dist == best_dist && f < best_f)) {
+      best_dist = dist;
+      best_f = f;
+      best_mask = mask;
+    }
+    if (s + 1 < cnt) {                              // flip free coordinate k = ctz(s+1)
+      const int k = __ffs(s + 1) - 1;
+      const float sg2 = ((f >> k) & 1) ? -2.f : 2.f;  // r_F moves by sg2 * M[:, d+k]
+      float mk[DM], pk[DM];
+      load_column<DM>(t.CM[d + k], mk);
+      load_column<DM>(t.CP[k], pk);
+      mask = 0;
+#pragma unroll
+      for (int i = 0; i < DM; ++i) {
+        rF[i] = fmaf(sg2, mk[i], rF[i]);
+        u[i] = fmaf(sg2, pk[i], u[i]);
+        if (i < d && u[i] < 0.f) mask |= 1u << i;
+      }
+      f ^= 1u << k;
+    }
+  }
+}
+
+template <int DM, bool kSeeded, bool kTable>
 __global__ void __launch_bounds__(kThreads, 4) encode_kernel(const Params p) {
   __shared__ Tables t;
+  extern __shared__ __align__(16) float Tsm[];   // kTable: M_S b_S for every solved sign pattern
   build_tables(p, t);
+  if (kTable) {
+    constexpr int DP = (DM + 3) / 4 * 4;
+    for (int e = threadIdx.x; e < (DP << p.d); e += blockDim.x) {
+      const int m = e / DP, i = e - m * DP;
+      float a = 0.f;
+      if (i < p.d)
+        for (int c = 0; c < p.d; ++c) a = fmaf(t.M[i][c], ((m >> c) & 1) ? -1.f : 1.f, a);
+      Tsm[e] = a;
+    }
+    __syncthreads();
+  }
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (int64_t)gridDim.x * kWarps;
   const int64_t ntask = p.N * p.G;
@@ -284,7 +365,9 @@ __global__ void __launch_bounds__(kThreads, 4) encode_kernel(const Params p) {
     for (int i = 0; i < DM; ++i) w[i] = __shfl_sync(0xffffffffu, mine, i);
     float bd;
     uint32_t bi, bmask = 0;
-    if (kSeeded)
+    if (kSeeded && kTable)
+      search_seeded_table<DM>(p, t, Tsm, w, lane, bd, bi, bmask);
+    else if (kSeeded)
       search_seeded<DM>(p, t, w, lane, bd, bi, bmask);
     else
       search_exact<DM>(p, t, w, lane, bd, bi);
@@ -319,15 +402,32 @@ __global__ void __launch_bounds__(kThreads, 4) encode_kernel(const Params p) {
   }
 }
 
+// the seeded search with the 2^d table, for d <= 10 (at most 48 KB of shared memory)
+template <int DM>
+static cudaError_t launch_table(const Params& p, int grid, cudaStream_t st) {
+  static int set[64];
+  const size_t bytes = (size_t)((DM + 3) / 4 * 4 << p.d) * sizeof(float);
+  cudaError_t e = ensure_smem((const void*)encode_kernel<DM, true, true>, bytes, set);
+  if (e != cudaSuccess) return e;
+  encode_kernel<DM, true, true><<<grid, kThreads, bytes, st>>>(p);
+  return cudaGetLastError();
+}
+
 template <bool kSeeded>
 static cudaError_t launch_mode(const Params& p, int grid, cudaStream_t st) {
   const int d = p.d;
-  if (d <= 2) encode_kernel<2, kSeeded><<<grid, kThreads, 0, st>>>(p);
-  else if (d <= 4) encode_kernel<4, kSeeded><<<grid, kThreads, 0, st>>>(p);
-  else if (d <= 8) encode_kernel<8, kSeeded><<<grid, kThreads, 0, st>>>(p);
-  else if (d <= 10) encode_kernel<10, kSeeded><<<grid, kThreads, 0, st>>>(p);
-  else if (d <= 12) encode_kernel<12, kSeeded><<<grid, kThreads, 0, st>>>(p);
-  else encode_kernel<16, kSeeded><<<grid, kThreads, 0, st>>>(p);
+  if (kSeeded && d <= 10) {
+    if (d <= 2) return launch_table<2>(p, grid, st);
+    if (d <= 4) return launch_table<4>(p, grid, st);
+    if (d <= 8) return launch_table<8>(p, grid, st);
+    return launch_table<10>(p, grid, st);
+  }
+  if (d <= 2) encode_kernel<2, kSeeded, false><<<grid, kThreads, 0, st>>>(p);
+  else if (d <= 4) encode_kernel<4, kSeeded, false><<<grid, kThreads, 0, st>>>(p);
+  else if (d <= 8) encode_kernel<8, kSeeded, false><<<grid, kThreads, 0, st>>>(p);
+  else if (d <= 10) encode_kernel<10, kSeeded, false><<<grid, kThreads, 0, st>>>(p);
+  else if (d <= 12) encode_kernel<12, kSeeded, false><<<grid, kThreads, 0, st>>>(p);
+  else encode_kernel<16, kSeeded, false><<<grid, kThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 
