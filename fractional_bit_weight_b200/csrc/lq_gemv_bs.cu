@@ -111,13 +111,17 @@ __device__ __forceinline__ void record_status(uint32_t* status, uint32_t code) {
   atomicCAS(status, 0u, code);
 }
 
-// Waits for the phase of `bar` with the given parity; false after kWaitNs.
+// Waits for the phase of `bar` with the given parity; false after kWaitNs. The clock is read
+// once per 32 tries, so that a waiting warp takes few issue slots from the others.
 __device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity) {
   if (sm100::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = gtime();
-  while (!sm100::mbar_try_wait(bar, parity))
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (sm100::mbar_try_wait(bar, parity)) return true;
     if (gtime() - t0 > bs::kWaitNs) return false;
-  return true;
+  }
 }
 
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -687,23 +691,10 @@ int bs_sm_count() {
   return cached[dev];
 }
 
-// Stage windows of a slice of sc chunks: an odd width of at most kMaxWindow chunks (a stage row
-// stride of 64 mod 128 bytes), the fewest chunks fetched past the slice, then the widest.
-int window_chunks(int sc) {
-  int best = 0, best_waste = 1 << 30;
-  const int n0 = (sc + bs::kMaxWindow - 1) / bs::kMaxWindow;
-  for (int nwin = n0; nwin <= n0 + 4; ++nwin) {
-    int w = (sc + nwin - 1) / nwin;
-    if (w % 2 == 0) ++w;
-    if (w > bs::kMaxWindow) continue;
-    const int waste = (sc + w - 1) / w * w - sc;
-    if (waste < best_waste || (waste == best_waste && w > best)) {
-      best = w;
-      best_waste = waste;
-    }
-  }
-  return best;
-}
+// Chunks fetched past a slice of sc chunks read in windows of w: past the last slice they lie
+// past the end of the row (the box reads zeros there, no traffic); inside they are the next
+// slice's bytes, read for nothing.
+int window_waste(int sc, int w) { return (sc + w - 1) / w * w - sc; }
 }  // namespace
 
 BsPlan plan_gemv_bs(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, int32_t D,
@@ -724,44 +715,52 @@ BsPlan plan_gemv_bs(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, i
   if (p.prep_smem > 200 * 1024) return p;
   const int sms = bs_sm_count();
   constexpr size_t kBudget = 224 * 1024;
-  for (int S = 1; S <= 16 && !p.ok; ++S) {
-    const int sc = (p.nchunk + S - 1) / S;
-    if (S > 1 && (p.nchunk + sc - 1) / sc != S) continue;   // no empty slice
-    const int R = std::max(1, std::min(sms / S, (N + 15) / 16));
-    const int rq = N / R;
-    const int rows_max = rq + 1;
-    const size_t frag = (size_t)sc * batch * bs::kTokBytes + bs::kZeroBytes;
-    const size_t acc_bytes = (size_t)rows_max * 8 * p.nt * 4;
-    const size_t fixed = frag + acc_bytes;
-    if (fixed > kBudget) continue;
-    const int wch = window_chunks(sc);
-    if (wch == 0) continue;
-    const int stride = 64 * wch;
-    int rs = 0, NS = 0;
-    for (int r : {32, 16}) {
-      const size_t stage = (size_t)r * stride;
-      const int ns = (int)std::min<size_t>((kBudget - fixed) / stage, bs::kMaxStages);
-      if (ns >= 3) {
-        rs = r;
-        NS = ns;
-        break;
+  // K-slices and stages: 32-row stages if any slicing leaves room for >= 3 of them, else 16-row
+  // ones; the fewest slices (their cross-slice sum costs more than wider stages gain); then the
+  // most useful bytes per stage (rows x the slice's chunks per window: the stage, not the byte,
+  // carries the fixed cost of the loop). A window is an odd number of chunks (a row stride of 64
+  // mod 128 bytes), at most kMaxWindow, at least 8 chunks where the slice has them; windows may
+  // run past a slice by at most 1/32 of it (at least one chunk) inside the row, freely past its
+  // end.
+  for (int r : {32, 16}) {
+    for (int S = 1; S <= 16 && !p.ok; ++S) {
+      const int sc = (p.nchunk + S - 1) / S;
+      if (S > 1 && (p.nchunk + sc - 1) / sc != S) continue;   // no empty slice
+      const int R = std::max(1, std::min(sms / S, (N + 15) / 16));
+      const int rq = N / R;
+      const int rows_max = rq + 1;
+      const size_t frag = (size_t)sc * batch * bs::kTokBytes + bs::kZeroBytes;
+      const size_t acc_bytes = (size_t)rows_max * 8 * p.nt * 4;
+      const size_t fixed = frag + acc_bytes;
+      if (fixed > kBudget) continue;
+      double best = 0.0;
+      for (int w = 1; w <= bs::kMaxWindow; w += 2) {
+        const int nwin = (sc + w - 1) / w;
+        if (S > 1 && window_waste(sc, w) > std::max(1, sc / 32)) continue;
+        const size_t stage = (size_t)r * 64 * w;
+        const int NS = (int)std::min<size_t>((kBudget - fixed) / stage, bs::kMaxStages);
+        if (NS < 3) continue;
+        const double useful = (double)sc / nwin;
+        if (useful < std::min(8, sc)) continue;   // box rows of >= 512 bytes stream at full rate
+        if (useful > best) {
+          best = useful;
+          p.S = S;
+          p.sc = sc;
+          p.R = R;
+          p.rq = rq;
+          p.rrem = N % R;
+          p.rows_max = rows_max;
+          p.rows_per_stage = r;
+          p.wch = w;
+          p.stride = 64 * w;
+          p.NS = NS;
+          p.frag_smem = frag;
+          p.smem = fixed + (size_t)NS * stage;
+          p.ok = true;
+        }
       }
     }
-    if (rs == 0) continue;
-    p.S = S;
-    p.sc = sc;
-    p.R = R;
-    p.rq = rq;
-    p.rrem = N % R;
-    p.rows_max = rows_max;
-    p.rows_per_stage = rs;
-    p.wch = wch;
-    p.stride = stride;
-    p.NS = NS;
-    p.frag_smem = frag;
-    p.smem = frag + (size_t)NS * rs * stride + acc_bytes;
-    p.ok = true;
-    break;
+    if (p.ok) break;
   }
   if (!p.ok) return p;
   p.nctas = p.S * p.R;
