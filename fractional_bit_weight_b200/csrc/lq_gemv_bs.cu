@@ -186,18 +186,21 @@ __device__ __forceinline__ float scale_from_bound(float cm, float a2) {
 }
 
 // This thread's part of the largest squared block norm of token t over all of K (identity T:
-// the largest x^2). With blocks of >= 8 inputs, lane l of warp w takes the 8 inputs from
-// 8 (32 w + l) + 2048 r in round r (the loads of four rounds in flight together) and the
-// Bh / 8 lanes of one block add their sums by shuffles. The caller reduces over the CTA.
-__device__ float prep_block_norms(const BsPrepParams& P, int t) {
+// the largest x^2). With blocks of >= 8 inputs, warps w0 .. w0 + nw - 1 share the pass: lane l
+// of the i-th of them takes the 8 inputs from 8 (32 i + l) + 256 nw r in round r (the loads of
+// four rounds in flight together) and the Bh / 8 lanes of one block add their sums by
+// shuffles. The caller reduces over the CTA.
+__device__ float prep_block_norms(const BsPrepParams& P, int t, int w0, int nw) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Bh = P.T.block;
   const int64_t off = (int64_t)t * P.K;
   float m = 0.f;
   if (Bh >= 8) {
-    // K is a multiple of Bh (<= 256), so a block's lanes are all in range or all out
+    // warps w0 .. w0 + nw - 1 only; K is a multiple of Bh (<= 256), so a block's lanes are all
+    // in range or all out
+    if (warp < w0 || warp >= w0 + nw) return 0.f;
 #pragma unroll 4
-    for (int kw = 8 * 32 * warp; kw < P.K; kw += 8 * bs::kPrepThreads) {
+    for (int kw = 8 * 32 * (warp - w0); kw < P.K; kw += 8 * 32 * nw) {
       const int k = kw + 8 * lane;
       const bool in = k < P.K;
       float v[8];
@@ -308,9 +311,16 @@ __global__ void __launch_bounds__(bs::kPrepThreads) gemv_bs_prep_kernel(const Bs
       }
     }
   }
-  // 2. every token's largest squared block norm over all of K
+  // 2. every token's largest squared block norm over all of K, by the warps that whitened
+  // nothing when that leaves at least half of them (their loads then go out with the
+  // whitening's instead of after them)
+  int w0 = 0;
+  if (Bh >= 32) {
+    const int tasks = P.batch * (span / Bh);
+    if (tasks <= bs::kPrepWarps / 2) w0 = tasks;
+  }
   for (int tok = 0; tok < P.batch; ++tok) {
-    const float m = bs_warp_max(prep_block_norms(P, tok));
+    const float m = bs_warp_max(prep_block_norms(P, tok, w0, bs::kPrepWarps - w0));
     if (lane == 0) s_red[tok][warp] = m;
   }
   __syncthreads();
