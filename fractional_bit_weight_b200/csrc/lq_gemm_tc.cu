@@ -10,9 +10,10 @@
 //    2^e chosen from a bound on |z|, written as fp16 z * 2^e. Inside every 32-coordinate word
 //    the coordinates are stored in the order q0, q0+16, q0+1, q0+17, ..., q0+15, q0+31 -- the
 //    order in which the GEMM unpacks a 32-bit code word into fp16 pairs (see pm1_pair).
-//  * gemm_tc_kernel (persistent, one CTA per SM): 128-token x 256-row output tiles, taken
-//    token tile fastest, so that the CTAs of one wave share the codes of a few row tiles in L2
-//    while the (smaller) z matrix stays resident there. A warp
+//  * gemm_tc_kernel (persistent, one CTA per SM): 128-token x 256-row output tiles, in groups
+//    of token tiles holding ~40 MB of z, each group swept across all row tiles token tile
+//    fastest: the group's z stays resident in L2 and the CTAs of one wave share the codes of a
+//    few row tiles; the codes are read once per group. A warp
 //    loads the fp16 z tile with TMA (128-byte swizzle); eight warps expand the stored bits of
 //    256 rows into +-1 fp16 in the same swizzled K-major layout; one thread issues
 //    tcgen05.mma (fp32 accumulation in tensor memory, two accumulators so the epilogue of one
@@ -74,7 +75,20 @@ struct TcArgs {
   float* y;
   uint32_t* status;         // workspace status word
   int N, batch, nks, tiles_n, tiles_m, tiles, sdt, vec_store;
+  int group_m;   // token tiles per raster group
 };
+
+// Tile -> (token tile, row tile): groups of group_m token tiles, each swept across every row
+// tile, token tile fastest inside a group. A group's z (group_m x 128 tokens) stays in L2 while
+// its row tiles stream past, and a wave of CTAs shares the codes of a few row tiles; the codes
+// are read once per group.
+__device__ __forceinline__ void tile_coords(const TcArgs& a, int tile, int& tm, int& tn) {
+  const int span = a.group_m * a.tiles_n;
+  const int grp = tile / span, r = tile - grp * span;
+  const int gm = min(a.group_m, a.tiles_m - grp * a.group_m);
+  tm = grp * a.group_m + r % gm;
+  tn = r / gm;
+}
 
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
@@ -160,7 +174,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- epilogue
     int lt = 0;
     for (int tile = blockIdx.x; tile < a.tiles; tile += gridDim.x, ++lt) {
-      const int tm = tile % a.tiles_m, tn = tile / a.tiles_m;
+      int tm, tn;
+      tile_coords(a, tile, tm, tn);
       const int b = lt & 1;
       // tcgen05.ld below is warp-collective: every lane must take the same branch here
       if (!__all_sync(0xffffffffu, wait_phase(&ctl->tmem_full[b], (lt >> 1) & 1, abort, true))) {
@@ -209,7 +224,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t ctr = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < a.tiles; tile += gridDim.x) {
-        const int tm = tile % a.tiles_m;
+        int tm, tn;
+        tile_coords(a, tile, tm, tn);
         for (int k = 0; k < a.nks; ++k, ++ctr) {
           const int slot = ctr % NSTAGE;
           if (!wait_phase(&ctl->empty[slot], ((ctr / NSTAGE) & 1) ^ 1, abort, true)) {
@@ -276,7 +292,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ctr = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < a.tiles; tile += gridDim.x) {
-      const int tn = tile / a.tiles_m;
+      int tm, tn;
+      tile_coords(a, tile, tm, tn);
       const int n = tn * BN + p;
       const bool valid = n < a.N;
       const uint2* rp = reinterpret_cast<const uint2*>(a.packed + (valid ? (int64_t)n * a.row_words : 0));
@@ -494,6 +511,8 @@ TcPlan plan_gemm_tc(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d) {
   p.tiles_n = (int)tn;
   p.tiles_m = (int)tm;
   p.tiles = (int)(tn * tm);
+  // token tiles per raster group: about 40 MB of fp16 z, a third of L2
+  p.group_m = (int)std::max<int64_t>(1, std::min<int64_t>(tm, (40ll << 20) / ((int64_t)tc::BM * Lp * 2)));
   p.smem = tc::kSmemBytes;
   p.z_bytes = (size_t)batch * Lp * sizeof(__half);
   p.scale_bytes = (size_t)batch * sizeof(float);
@@ -546,6 +565,7 @@ cudaError_t launch_gemm_tc(const TcPlan& pl, const void* x, int xdt, int32_t bat
   a.tiles_n = pl.tiles_n;
   a.tiles_m = pl.tiles_m;
   a.tiles = pl.tiles;
+  a.group_m = pl.group_m;
   a.sdt = sdt;
   a.vec_store = (N % 4 == 0) && (reinterpret_cast<uintptr_t>(y) % 16 == 0);
   const int grid = std::min(pl.tiles, sms);

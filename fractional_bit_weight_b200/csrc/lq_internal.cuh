@@ -93,6 +93,7 @@ struct TcPlan {
   int Lp;              // lifted length padded to the 64-coordinate stage
   int nks;             // stages per tile (Lp / 64)
   int tiles_n, tiles_m, tiles;
+  int group_m;         // token tiles per raster group
   size_t smem;         // GEMM dynamic shared memory per CTA
   size_t pro_smem;     // prologue dynamic shared memory per CTA
   size_t z_bytes;      // scratch: fp16 z [batch][Lp]
