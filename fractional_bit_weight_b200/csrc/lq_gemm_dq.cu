@@ -7,8 +7,8 @@
 // reading W once (2 bytes per weight). Three kernels:
 //
 //  * dq_weights_kernel: W[n][g*d + i] = sum_j M[i][j] b[n][g][j] for every block g of every
-//    row, on the legacy tensor cores (mma.m16n8k16, fp32 accumulation): A is M (rows i, columns
-//    j) rounded to fp16, B the +-1 codes of eight blocks (columns), +-1 being exact in fp16.
+//    row, on the legacy tensor cores (mma.m16n8k16, fp32 accumulation): A holds the +-1 codes of
+//    sixteen blocks (rows), exact in fp16, B is M^T (columns i) rounded to fp16.
 //    The rounding of M adds at most 2^-12 of each |M[i][j]| to a sum of D such terms, about as
 //    much as the final rounding of W to fp16 (relative 2^-12); with the fp16 rounding of T(x)
 //    the expected relative error of y is ~3e-4, against the 2e-3 tolerance. Columns from Kp to
@@ -261,39 +261,48 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
 }
 
 constexpr int kDqWarps = 16;
-constexpr int kDqSets = 16;   // sets of 8 blocks per flush of the W staging buffer
+constexpr int kDqGroups = 8;   // groups of 16 blocks per flush of the W staging buffer
 
 // One warp per row (grid-stride over rows): the row's code words are copied to shared memory
-// with coalesced 16-byte loads, then sets of 8 blocks go through the MMAs (each lane reads its
-// block's bits from shared memory); the fp16 results of kDqSets sets gather in a shared-memory
-// piece of the W row, which the warp writes out with coalesced 16-byte stores. d <= 16, D <= 32.
-// Dynamic shared memory per warp: the row's code words + 16 bytes, then kDqSets * 8 * d fp16.
+// with coalesced 16-byte loads, then groups of 16 blocks go through the MMAs as C = A B, A the
+// +-1 codes (16 blocks x 16 code positions, exact in fp16), B = M^T (16 code positions x 8 rows
+// i of a block; a second column tile when d > 8), so a lane holds two consecutive outputs i of
+// two blocks. They gather as fp16 pairs in a shared-memory piece of the W row, which the warp
+// writes out with coalesced 16-byte stores. d <= 16, D <= 32. Dynamic shared memory per warp:
+// the row's code words + 16 bytes, then kDqGroups * 16 * d fp16.
+template <int NKS>
 __global__ void __launch_bounds__(kDqWarps * 32)
     dq_weights_kernel(const uint32_t* __restrict__ packed, int64_t row_words, int N, int G,
                       const float* __restrict__ M, int d, int D, int Kw, __half* __restrict__ W) {
   extern __shared__ __align__(16) uint8_t dsm[];
+  // fp16 +-1 pairs for the four values of two code bits (bit 1 is -1, the fp16 sign bit); the
+  // lanes read different entries, four words on four banks
+  __shared__ uint32_t pm1_pairs[4];
+  if (threadIdx.x < 4)
+    pm1_pairs[threadIdx.x] = ((threadIdx.x & 1u) << 15) | ((threadIdx.x >> 1) << 31) | 0x3C003C00u;
+  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const size_t code_bytes = ((size_t)row_words * 4 + 16 + 15) / 16 * 16;
-  const size_t piece = (size_t)kDqSets * 8 * d;            // fp16 per flush
-  uint8_t* mine = dsm + (size_t)warp * (code_bytes + piece * 2);
-  uint32_t* sc = reinterpret_cast<uint32_t*>(mine);                  // the row's code words
-  __half* sw = reinterpret_cast<__half*>(mine + code_bytes);         // a piece of the W row
-  // A fragments of M (rows i, columns j) in fp16, k-steps of 16 columns
-  uint32_t ah[2][4];
+  const size_t piece = (size_t)kDqGroups * 16 * d;           // fp16 per flush
+  uint8_t* mine = dsm + (size_t)warp * (code_bytes + (piece * 2 + 15) / 16 * 16);
+  uint32_t* sc = reinterpret_cast<uint32_t*>(mine);
+  __half* sw = reinterpret_cast<__half*>(mine + code_bytes);
+  // B fragments of M^T: B[j][i] = M[i][j], j = 16 ks + 2t (+1), + 8 (+1); i = g + 8 nt
+  uint32_t bm[NKS][2][2];
 #pragma unroll
-  for (int ks = 0; ks < 2; ++ks)
+  for (int ks = 0; ks < NKS; ++ks)
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int i = g + 8 * (r & 1);
-      const int j = 16 * ks + 2 * t + 8 * (r >> 1);
-      float m0 = 0.f, m1 = 0.f;
-      if (i < d && j < D) m0 = M[i * D + j];
-      if (i < d && j + 1 < D) m1 = M[i * D + j + 1];
-      ah[ks][r] = pack_h2(m0, m1);
-    }
-  const int nks = D > 16 ? 2 : 1;
-  const int nsets = (G + 7) / 8;
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int i = g + 8 * nt, j = 16 * ks + 2 * t + 8 * h;
+        float m0 = 0.f, m1 = 0.f;
+        if (i < d && j < D) m0 = M[i * D + j];
+        if (i < d && j + 1 < D) m1 = M[i * D + j + 1];
+        bm[ks][nt][h] = pack_h2(m0, m1);
+      }
+  const int ngrp = (G + 15) / 16;
   const int row_u4 = (int)(row_words / 4);                 // rows are 16-byte multiples
   const int gw = blockIdx.x * kDqWarps + warp, nw = gridDim.x * kDqWarps;
   for (int n = gw; n < N; n += nw) {
@@ -302,35 +311,57 @@ __global__ void __launch_bounds__(kDqWarps * 32)
     if (lane == 0) reinterpret_cast<uint4*>(sc)[row_u4] = make_uint4(0u, 0u, 0u, 0u);
     __syncwarp();
     __half* wrow = W + (int64_t)n * Kw;
-    for (int s0 = 0; s0 < nsets; s0 += kDqSets) {
-      for (int set = s0; set < min(nsets, s0 + kDqSets); ++set) {
-        const int blk = set * 8 + g;                       // this lane's block (B column g)
-        uint32_t bits = 0;
-        if (blk < G) {
-          const int q = blk * D;
-          const uint64_t win = (uint64_t)sc[(q >> 5) + 1] << 32 | sc[q >> 5];
-          bits = (uint32_t)(win >> (q & 31));
+    for (int g0 = 0; g0 < ngrp; g0 += kDqGroups) {
+      for (int gr = g0; gr < min(ngrp, g0 + kDqGroups); ++gr) {
+        // the lane's blocks: rows g and g + 8 of A (blocks past G give zero codes)
+        const int blk0 = gr * 16 + g, blk1 = blk0 + 8;
+        uint32_t bits0 = 0, bits1 = 0;
+        if (blk0 < G) {
+          const int q = blk0 * D;
+          bits0 = (uint32_t)(((uint64_t)sc[(q >> 5) + 1] << 32 | sc[q >> 5]) >> (q & 31));
         }
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        if (blk1 < G) {
+          const int q = blk1 * D;
+          bits1 = (uint32_t)(((uint64_t)sc[(q >> 5) + 1] << 32 | sc[q >> 5]) >> (q & 31));
+        }
+        bits0 >>= 2 * t;
+        bits1 >>= 2 * t;
+        float c[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-          if (ks < nks) {
-            const uint32_t b0 = pm1_h2(bits, 16 * ks + 2 * t);
-            const uint32_t b1 = pm1_h2(bits, 16 * ks + 2 * t + 8);
-            hmma_16816(c, ah[ks], b0, b1);
+        for (int ks = 0; ks < NKS; ++ks) {
+          // code positions 16 ks + 2t (+1) and + 8 (+1); positions >= D meet zero rows of B, so
+          // the bits past a block (the next block's) do not matter
+          uint32_t a[4];
+          a[0] = pm1_pairs[(bits0 >> (16 * ks)) & 3u];
+          a[1] = pm1_pairs[(bits1 >> (16 * ks)) & 3u];
+          a[2] = pm1_pairs[(bits0 >> (16 * ks + 8)) & 3u];
+          a[3] = pm1_pairs[(bits1 >> (16 * ks + 8)) & 3u];
+          hmma_16816(c[0], a, bm[ks][0][0], bm[ks][0][1]);
+          if (d > 8) hmma_16816(c[1], a, bm[ks][1][0], bm[ks][1][1]);
+        }
+        // C[blk][i]: this lane holds (blk0, i0), (blk0, i0 + 1), (blk1, i0), (blk1, i0 + 1)
+        __half* pw = sw + (size_t)(gr - g0) * 16 * d;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const int i0 = 8 * nt + 2 * t;
+          if (i0 >= d) continue;
+#pragma unroll
+          for (int hb = 0; hb < 2; ++hb) {
+            const int col = (g + 8 * hb) * d + i0;
+            const float lo = c[nt][2 * hb], hi = c[nt][2 * hb + 1];
+            if (i0 + 1 < d && (col & 1) == 0) {
+              *reinterpret_cast<uint32_t*>(pw + col) = pack_h2(lo, hi);
+            } else {
+              pw[col] = __float2half_rn(lo);
+              if (i0 + 1 < d) pw[col + 1] = __float2half_rn(hi);
+            }
           }
-        }
-        // C[i][col]: this lane holds (g, 2t), (g, 2t+1), (g+8, 2t), (g+8, 2t+1)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int i = g + 8 * (r >> 1), col = 2 * t + (r & 1);
-          if (i < d) sw[((set - s0) * 8 + col) * d + i] = __float2half_rn(c[r]);
         }
       }
       __syncwarp();
-      // the piece covers W columns [s0*8*d, ...): blocks past G give columns >= G*d, which
+      // the piece covers W columns [g0*16*d, ...): blocks past G give columns >= G*d, which
       // must read zero; columns past Kw are not written
-      const int k0 = s0 * 8 * d;
+      const int k0 = g0 * 16 * d;
       const int kend = min(Kw, k0 + (int)piece);
       for (int k = k0 + 8 * lane; k < kend; k += 256) {
         uint4 v = *reinterpret_cast<const uint4*>(sw + (k - k0));
@@ -344,8 +375,8 @@ __global__ void __launch_bounds__(kDqWarps * 32)
       }
       __syncwarp();
     }
-    // columns past the last piece (Kw > nsets * 8 * d happens only through the 64 padding)
-    for (int k = max(nsets * 8 * d, 0) + 8 * lane; k < Kw; k += 256)
+    // columns past the last piece (the padding to the 64-input stage)
+    for (int k = ngrp * 16 * d + 8 * lane; k < Kw; k += 256)
       *reinterpret_cast<uint4*>(wrow + k) = make_uint4(0u, 0u, 0u, 0u);
     __syncwarp();
   }
@@ -429,7 +460,7 @@ DqPlan plan_gemm_dq(int32_t batch, int32_t N, int32_t K, int32_t d, int32_t D) {
   // the dequantisation kernel: per warp the row's code words (+16 bytes) and a piece of W
   const int64_t row_bytes = ((G * D + 7) / 8 + 15) / 16 * 16;
   p.dq_smem = (size_t)dq::kDqWarps * ((size_t)(row_bytes + 16 + 15) / 16 * 16 +
-                                      (size_t)dq::kDqSets * 8 * d * 2);
+                                      ((size_t)dq::kDqGroups * 16 * d * 2 + 15) / 16 * 16);
   if (p.dq_smem > 220 * 1024) return p;
   p.dq_ctas_per_sm = (int)std::max<size_t>(1, std::min<size_t>(2, 220 * 1024 / p.dq_smem));
   p.xt_smem = (size_t)K * sizeof(float);
@@ -444,7 +475,7 @@ cudaError_t launch_gemm_dq(const DqPlan& pl, const void* x, int xdt, int32_t bat
                            Whiten T, const float* M, int32_t d, int32_t D,
                            const uint32_t* packed, int64_t row_bytes, int32_t N, const void* s,
                            int sdt, float* y, void* scratch, uint32_t* status, cudaStream_t st) {
-  static int xt_set[64], gemm_set[64], dq_set[64];
+  static int xt_set[64], gemm_set[64], dq_set[64], dq_set1[64];
   uint8_t* sp = static_cast<uint8_t*>(scratch);
   __half* W = reinterpret_cast<__half*>(sp);
   __half* xh = reinterpret_cast<__half*>(sp + pl.w_bytes);
@@ -452,12 +483,17 @@ cudaError_t launch_gemm_dq(const DqPlan& pl, const void* x, int xdt, int32_t bat
   const int sms = tc_sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
 
-  cudaError_t e = ensure_smem((const void*)dq::dq_weights_kernel, pl.dq_smem, dq_set);
+  const void* dqk = D > 16 ? (const void*)dq::dq_weights_kernel<2> : (const void*)dq::dq_weights_kernel<1>;
+  cudaError_t e = ensure_smem(dqk, pl.dq_smem, D > 16 ? dq_set : dq_set1);
   if (e != cudaSuccess) return e;
   const int dq_ctas = (int)std::min<int64_t>((int64_t)sms * pl.dq_ctas_per_sm,
                                              (N + dq::kDqWarps - 1) / dq::kDqWarps);
-  dq::dq_weights_kernel<<<dq_ctas, dq::kDqWarps * 32, pl.dq_smem, st>>>(packed, row_bytes / 4, N,
-                                                                      pl.G, M, d, D, pl.Kw, W);
+  if (D > 16)
+    dq::dq_weights_kernel<2><<<dq_ctas, dq::kDqWarps * 32, pl.dq_smem, st>>>(
+        packed, row_bytes / 4, N, pl.G, M, d, D, pl.Kw, W);
+  else
+    dq::dq_weights_kernel<1><<<dq_ctas, dq::kDqWarps * 32, pl.dq_smem, st>>>(
+        packed, row_bytes / 4, N, pl.G, M, d, D, pl.Kw, W);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = ensure_smem((const void*)dq::xt_f16_kernel, pl.xt_smem, xt_set);
