@@ -321,9 +321,8 @@ int32_t lq_gemm_launches(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t
   if (!valid_code(K, d, D) || batch < 1 || batch > kMaxBatch || N < 1 || K > kMaxK) return 0;
   if (block < 0 || block > LQ_MAX_HADAMARD || (block & (block - 1)) != 0) return 0;
   const WsLayout lay = layout_gemm(batch, K, N, d, D, block);
-  // path 4: one kernel; paths 0 and 2: a prologue kernel and a contraction kernel, per token
-  // group on path 3; path 1: nothing (the call is rejected)
-  if (lay.path == 4) return 2;
+  // paths 0, 2 and 4: a prologue kernel and a contraction kernel, per token group on path 3;
+  // path 5: three; path 1: nothing (the call is rejected)
   if (lay.path == 1) return 0;
   if (lay.path == 5) return 3;   // W, xt, GEMM
   return lay.path == 3 ? 2 * ((batch + lay.gs - 1) / lay.gs) : 2;

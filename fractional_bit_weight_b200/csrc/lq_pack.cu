@@ -1,8 +1,8 @@
 // lq_pack.cu -- sign codes <-> LQ_FORMAT_V1 rows (offline step; not on the decode path).
 //
 // Paper (sec. 3.1): every length-d block is w ~= M w_q with w_q in {+1,-1}^D; the D signs of
-// block g of row n are stored as bits g*D .. g*D+D-1 of the row, a set bit meaning -1, so
-// the bit is exactly the IEEE sign bit that the decode kernels XOR onto z.
+// block g of row n are stored as bits g*D .. g*D+D-1 of the row, a set bit meaning -1 (the
+// value of the IEEE sign bit of the +-1 it stands for).
 #include "lq_internal.cuh"
 
 namespace lq {
