@@ -59,7 +59,7 @@ def test_codebook_rounds_match_oracle(orc, d, D, mode, S):
         mses.append(mse_g)
         print(f"d={d} D={D} mode={mode} round {rnd}: codes equal {same:.4f}, mse {mse_g:.6f}")
     NOTES.append(f"codebook fit d={d} D={D} {'seeded' if mode == lq.LQ_ENCODE_SEEDED else 'exact'} "
-                 f"S={S}: per-coordinate MSE of rounds 1-3 (round 1 = random M) " +
+                 f"S={S}: per-coordinate MSE of the encodings in three fit steps (the first under the random M) " +
                  ", ".join(f"{m:.5f}" for m in mses))
 
 
