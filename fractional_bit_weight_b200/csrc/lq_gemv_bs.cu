@@ -21,7 +21,7 @@
 //     memory with one bulk copy per token, then take the (stage rows, 64-byte chunk) items of
 //     each stage in turn: one AND per code word gives the int8 A operand (bit p of each byte as
 //     0 or 2^p) and the B entries carry 2^-p, so all eight bit positions accumulate into int32
-//     sums (up to four chains by bit position), exact across the whole row (a row of <= 2^17
+//     sums (two chains by bit-position parity), exact across the whole row (a row of <= 2^17
 //     coordinates cannot overflow); at the end of a row group each warp adds its sums into the
 //     CTA's per-row totals (integer shared-memory atomics, exact in any order). A stage row is
 //     a whole number of chunks, an odd one, so its stride is 64 mod 128 bytes and the two rows
@@ -467,7 +467,9 @@ __device__ __forceinline__ void run_window(int first, int nitems, uint32_t fwin,
 template <int NT, int HT>
 __global__ void __launch_bounds__(bs::kThreads, 1)
     gemv_bs_kernel(const __grid_constant__ CUtensorMap tmap, const BsParams P) {
-  constexpr int CH = NT == 1 ? 4 : NT == 2 ? 2 : 1;   // accumulator chains per (tile, B tile)
+  // accumulator chains per (tile, B tile): two chains by bit-position parity for one or two B
+  // tiles (four measured slower: more registers and more adds in every flush)
+  constexpr int CH = NT <= 2 ? 2 : 1;
   constexpr int RS = 16 * HT;           // rows per stage
   extern __shared__ __align__(1024) uint8_t smem[];
   __shared__ __align__(8) uint64_t full_bar[bs::kMaxStages], empty_bar[bs::kMaxStages];
