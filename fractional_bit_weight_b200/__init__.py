@@ -29,7 +29,7 @@ _DTYPES = {torch.float32: LQ_F32, torch.float16: LQ_F16, torch.bfloat16: LQ_BF16
 
 EXPORTS = ("lq_abi_version", "lq_lifted_bits", "lq_row_stride_bytes", "lq_pack", "lq_unpack", "lq_encode",
            "lq_whiten", "lq_lift", "lq_gemm_workspace_bytes", "lq_gemm_launches", "lq_gemm_route",
-           "lq_gemm", "lq_gemm_on_route", "lq_gemm_route_workspace_bytes",
+           "lq_gemm", "lq_gemm_on_route", "lq_gemm_route_workspace_bytes", "lq_gemv_staged_plan",
            "lq_codebook_workspace_bytes", "lq_codebook_round",
            "lq_gemm_noalloc", "lq_check_wait_timeout",
            "lq_device_status", "lq_status_string", "lq_last_error")
@@ -69,6 +69,7 @@ def _declare(L):
         "lq_gemm_on_route": ([vp, ctypes.c_int, i32, dp, vp, vp, vp, ctypes.c_int, i32, i32, i32,
                               i32, vp, vp, sz, i32, vp], ctypes.c_int),
         "lq_gemm_route_workspace_bytes": ([i32, i32, i32, i32, i32, i32, i32], sz),
+        "lq_gemv_staged_plan": ([i32, i32, i32, i32, i32, i32, ctypes.POINTER(i64)], ctypes.c_int),
         "lq_codebook_workspace_bytes": ([ctypes.c_int64, i32, i32], sz),
         "lq_codebook_round": ([vp, ctypes.c_int64, vp, i32, i32, i32, vp, vp, vp, sz, vp],
                               ctypes.c_int),
@@ -207,6 +208,17 @@ def lift(x, M, d, D, sign=None, chan_scale=None, block=0, out=None, stream=None)
 
 def gemm_workspace_bytes(batch, K, N, d, D):
     return int(lib().lq_gemm_workspace_bytes(batch, K, N, d, D))
+
+
+STAGED_PLAN_FIELDS = ("ok", "S", "sc", "R", "rq", "rrem", "rows_per_stage", "wch", "NS", "nchunk",
+                      "smem", "prep_smem")
+
+
+def gemv_staged_plan(batch, K, N, d, D, block=0):
+    """The TMA-staged GEMV's plan for a shape (host-only query), as a dict."""
+    out = (ctypes.c_int64 * len(STAGED_PLAN_FIELDS))()
+    _check(lib().lq_gemv_staged_plan(batch, K, N, d, D, block, out), "lq_gemv_staged_plan")
+    return dict(zip(STAGED_PLAN_FIELDS, (int(v) for v in out)))
 
 
 def gemm_launches(batch, K, N, d, D, block=0):

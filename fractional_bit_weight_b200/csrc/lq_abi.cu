@@ -328,6 +328,22 @@ int32_t lq_gemm_launches(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t
   return lay.path == 3 ? 2 * ((batch + lay.gs - 1) / lay.gs) : 2;
 }
 
+lq_status lq_gemv_staged_plan(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D,
+                              int32_t block, int64_t* out) {
+  clear_error();
+  if (out == nullptr) return fail(LQ_EINVAL, "null out");
+  if (!valid_code(K, d, D) || batch < 1 || batch > kMaxBatch || N < 1 || K > kMaxK)
+    return fail(LQ_EINVAL, "invalid sizes batch=%d K=%d N=%d d=%d D=%d", batch, K, N, d, D);
+  if (block < 0 || block > LQ_MAX_HADAMARD || (block & (block - 1)) != 0)
+    return fail(LQ_EINVAL, "invalid Hadamard block %d", block);
+  const lq::BsPlan p = lq::plan_gemv_bs(batch, lifted_bits(K, d, D), N, K, d, D, block);
+  const int64_t v[LQ_STAGED_PLAN_FIELDS] = {p.ok ? 1 : 0, p.S, p.sc, p.R, p.rq, p.rrem,
+                                            p.rows_per_stage, p.wch, p.NS, p.nchunk,
+                                            (int64_t)p.smem, (int64_t)p.prep_smem};
+  for (int i = 0; i < LQ_STAGED_PLAN_FIELDS; ++i) out[i] = v[i];
+  return LQ_OK;
+}
+
 int32_t lq_gemm_route(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D,
                       int32_t block) {
   if (!valid_code(K, d, D) || batch < 1 || batch > kMaxBatch || N < 1 || K > kMaxK) return -1;

@@ -204,6 +204,17 @@ LQ_API lq_status lq_gemm_on_route(const void* x, lq_dtype xdt, int32_t batch,
 LQ_API size_t lq_gemm_route_workspace_bytes(int32_t batch, int32_t K, int32_t N, int32_t d,
                                             int32_t D, int32_t block, int32_t route);
 
+/* The plan of the TMA-staged GEMV (LQ_ROUTE_GEMV_BULK) for this shape and Hadamard block.
+ * Host-only, touches no device; no counterpart on the pages: it lets tests check the plan's
+ * coverage and bounds. out[0 .. LQ_STAGED_PLAN_FIELDS) receives: ok (0: no staged plan fits),
+ * K-slices S, chunks per slice, row ranges R, rows per range (ranges 0 .. rrem-1 take one more),
+ * rrem, rows per stage, chunks per window, ring stages, 512-coordinate chunks per row, dynamic
+ * shared memory of the contraction kernel and of the prep kernel (bytes).
+ * Errors: LQ_EINVAL on invalid sizes or a null out. */
+#define LQ_STAGED_PLAN_FIELDS 12
+LQ_API lq_status lq_gemv_staged_plan(int32_t batch, int32_t K, int32_t N, int32_t d, int32_t D,
+                                     int32_t block, int64_t* out);
+
 /* Bytes of the scratch array that lq_gemm_noalloc keeps on every device that loads the library. */
 #define LQ_NOALLOC_SCRATCH_BYTES (8u << 20)
 
