@@ -11,18 +11,21 @@
 //    largest column 1-norm of M), so every chunk of a token shares one S; the whitening of the
 //    Hadamard blocks that feed the chunk; the lift z = M^T xt per block of d inputs (a lane
 //    keeps one column of M in registers and reads a block's inputs as broadcast loads); three
-//    int8 planes (base 254) of z * S * 2^-p, p = q mod 8, stored in the register layout of the
-//    B operand of mma.m16n8k32; and the chunk's sum of z.
+//    int8 planes (base 254) of the B operand of mma.m16n8k32 per bit slot of a code byte (see
+//    the item below), stored in its register layout; and the chunk's sum of z.
 //  gemv, S K-slices x R row ranges, one CTA per SM:
 //   * one producer thread streams the CTA's rows into a ring of shared-memory stages (32 or 16
 //     rows x a window of an odd number of 64-byte chunks) with 2-D TMA boxes of 8 rows. The
 //     codes are inputs of the call, so the stream starts at once, while the prep still runs;
 //   * the 16 compute warps wait for the prep grid, copy their slice's fragments into shared
 //     memory with one bulk copy per token, then take the (stage rows, 64-byte chunk) items of
-//     each stage in turn: one AND per code word gives the int8 A operand (bit p of each byte as
-//     0 or 2^p) and the B entries carry 2^-p, so all eight bit positions accumulate into int32
-//     sums (two chains by bit-position parity), exact across the whole row (a row of <= 2^17
-//     coordinates cannot overflow); at the end of a row group each warp adds its sums into the
+//     each stage in turn. A code byte v holds bits b_0..b_7 of eight coordinates; eight MMAs
+//     per byte take as A the raw byte read as unsigned (slot 0) and as signed (slot 7: it
+//     differs by 256 b_7) and, after one AND per code word, 2^q b_q alone (slots 1-6). The
+//     prep picks the slots' B entries so that the eight products weigh bit p by z_p S (up to
+//     rounding), and all slots accumulate into int32 sums (two chains by slot parity), exact
+//     across the whole row: a byte adds at most 127 (255 + 128 + 126) per digit plane, so a row
+//     of <= 2^17 coordinates stays below 2^31. At the end of a row group each warp adds its sums into the
 //     CTA's per-row totals (integer shared-memory atomics, exact in any order). A stage row is
 //     a whole number of chunks, an odd one, so its stride is 64 mod 128 bytes and the two rows
 //     of a quarter-warp's 16-byte loads fall on disjoint banks;
@@ -145,12 +148,20 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   return v;
 }
 
+// A as unsigned bytes (kSigned: as signed bytes), B signed bytes, int32 accumulators
+template <bool kSigned = false>
 __device__ __forceinline__ void imma(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                      uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};\n"
-      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  if (kSigned)
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  else
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ float bs_warp_max(float v) {
@@ -165,13 +176,21 @@ __device__ __forceinline__ float bs_warp_sum(float v) {
   return v;
 }
 
-// three int8 planes of base 254: a ~= P0 + P1/254 + P2/254^2 (|a| <= 64)
-__device__ __forceinline__ void bs_planes3(float a, int (&P)[3]) {
-  P[0] = __float2int_rn(a);
-  float r = (a - (float)P[0]) * 254.f;
-  P[1] = __float2int_rn(r);
-  r = (r - (float)P[1]) * 254.f;
-  P[2] = __float2int_rn(r);
+// z * S * 2^-p in units of 254^-2, rounded to the nearest integer (|z| * S < 64: below 2^22)
+__device__ __forceinline__ int bs_units(float zs, int p) {
+  return __float2int_rn(zs * __int_as_float((127 - p) << 23) * 64516.f);
+}
+
+// the three balanced base-254 digits of an integer c: c = 254^2 P0 + 254 P1 + P2, P1 and P2 in
+// [-127, 126] (|c| < 2^23: |P0| <= 128 / 1.27)
+__device__ __forceinline__ void bs_digits3(int c, int (&P)[3]) {
+  int q = c + 127;
+  q = q >= 0 ? q / 254 : -((253 - q) / 254);   // floor
+  P[2] = c - 254 * q;
+  int r = q + 127;
+  r = r >= 0 ? r / 254 : -((253 - r) / 254);
+  P[1] = q - 254 * r;
+  P[0] = r;
 }
 
 // The power-of-two scale S of a token from the largest squared Hadamard-block norm a2 of
@@ -389,19 +408,30 @@ __global__ void __launch_bounds__(bs::kPrepThreads) gemv_bs_prep_kernel(const Bs
     for (int w = 0; w < bs::kPrepWarps; ++w) a += s_sum[tid][w];
     P.csum[(int64_t)c * P.batch + tid] = a;
   }
-  // 4. quantise: thread -> (token, group of the B-operand layout), group -> (p, tt, h, j); its
-  // 4 coordinates e0 + 8 i fill one word per plane
+  // 4. quantise: thread -> (token, group of the B-operand layout), group -> (slot, tt, h, j); its
+  // 4 bytes e0 / 8 + i fill one word per plane. With I_p the code bit p's value z * S * 2^-p in
+  // units of 254^-2, a byte's eight products come from six masked bytes (slots 1-6: B = I_q -
+  // I_0) and the raw byte read twice: unsigned (slot 0, B = h) and signed (slot 7, B = I_0 - h),
+  // h = (I_0 + I_7) / 2. Bit 0 then weighs I_0, bit q 2^q I_q and bit 7 128 (2h - I_0) = 2^7 I_7.
   for (int it = tid; it < P.batch * 128; it += bs::kPrepThreads) {
     const int tok = it >> 7, grp = it & 127;
     const int pl8 = grp & 7, tt = (grp >> 3) & 3, hl = (grp >> 5) & 1, jl = grp >> 6;
-    const int e0 = 128 * tt + 64 * jl + 32 * hl + pl8;
-    const float Sp = s_tok[tok] * __int_as_float((127 - pl8) << 23);   // S * 2^-p, exact
+    const int e0 = 128 * tt + 64 * jl + 32 * hl;      // bit 0 of the group's first byte
+    const float S = s_tok[tok];
     uint32_t w4[bs::kPlanes] = {};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int e = e0 + 8 * i;
+      const float* zb = zc + tok * bs::kZc + (e0 + 8 * i) + ((e0 + 8 * i) >> 7) * 8;
+      // I_0 rounds to the nearest integer of I_7's parity (one unit at most), so that h is
+      // exact and bit 7 weighs I_7 itself: an odd sum would bias every set bit 7 by -128 units
+      const int I7 = bs_units(zb[7] * S, 7);
+      const float t0 = zb[0] * S * 64516.f;
+      int I0 = __float2int_rn(t0);
+      if ((I0 ^ I7) & 1) I0 += t0 > (float)I0 ? 1 : -1;
+      const int h = (I0 + I7) >> 1;
+      const int cq = pl8 == 0 ? h : pl8 == 7 ? I0 - h : bs_units(zb[pl8] * S, pl8) - I0;
       int Pq[bs::kPlanes];
-      bs_planes3(zc[tok * bs::kZc + e + (e >> 7) * 8] * Sp, Pq);
+      bs_digits3(cq, Pq);
 #pragma unroll
       for (int pl = 0; pl < bs::kPlanes; ++pl) w4[pl] |= ((uint32_t)Pq[pl] & 0xffu) << (8 * i);
     }
@@ -434,7 +464,8 @@ __device__ __forceinline__ void run_item(uint32_t arow, int stride, uint32_t fb,
     for (int e = 0; e < 2; ++e) {
       const int mma = 2 * m2 + e;
       const int j = mma >> 3, p = mma & 7;
-      const uint32_t msk = 0x01010101u << p;
+      // slots 0 and 7 take the raw bytes (unsigned, signed), slots 1-6 bit p alone
+      const uint32_t msk = (p == 0 || p == 7) ? 0xffffffffu : 0x01010101u << p;
       const int ch = CH == 4 ? 2 * (m2 & 1) + e : CH == 2 ? e : 0;
 #pragma unroll
       for (int h = 0; h < HA; ++h) {
@@ -443,7 +474,10 @@ __device__ __forceinline__ void run_item(uint32_t arow, int stride, uint32_t fb,
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const uint32_t b0 = e ? bv[nt].z : bv[nt].x, b1 = e ? bv[nt].w : bv[nt].y;
-          imma(acc[nt][h][ch], a0, a1, a2, a3, b0, b1);
+          if (p == 7)
+            imma<true>(acc[nt][h][ch], a0, a1, a2, a3, b0, b1);
+          else
+            imma(acc[nt][h][ch], a0, a1, a2, a3, b0, b1);
         }
       }
     }
