@@ -209,7 +209,8 @@ __device__ __forceinline__ float scale_from_bound(float cm, float a2) {
 // of the i-th of them takes the 8 inputs from 8 (32 i + l) + 256 nw r in round r (the loads of
 // four rounds in flight together) and the Bh / 8 lanes of one block add their sums by
 // shuffles. The caller reduces over the CTA.
-__device__ float prep_block_norms(const BsPrepParams& P, int t, int w0, int nw) {
+template <int XDT>
+__device__ __forceinline__ float prep_block_norms(const BsPrepParams& P, int t, int w0, int nw) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Bh = P.T.block;
   const int64_t off = (int64_t)t * P.K;
@@ -223,7 +224,7 @@ __device__ float prep_block_norms(const BsPrepParams& P, int t, int w0, int nw) 
       const int k = kw + 8 * lane;
       const bool in = k < P.K;
       float v[8];
-      load8_as_f32(P.x, P.xdt, off + (in ? k : 0), 8, v);
+      load8_as_f32(P.x, XDT, off + (in ? k : 0), 8, v);
       if (P.T.chan_scale) {
         float cs[8];
 #pragma unroll
@@ -242,7 +243,7 @@ __device__ float prep_block_norms(const BsPrepParams& P, int t, int w0, int nw) 
       float a = 0.f;
       for (int i = 0; i < Bh; ++i) {
         const int k = b * Bh + i;
-        float v = load_as_f32(P.x, P.xdt, off + k);
+        float v = load_as_f32(P.x, XDT, off + k);
         if (P.T.chan_scale) v *= __ldg(P.T.chan_scale + k);
         a = fmaf(v, v, a);
       }
@@ -250,7 +251,7 @@ __device__ float prep_block_norms(const BsPrepParams& P, int t, int w0, int nw) 
     }
   } else {
     for (int k = tid; k < P.K; k += bs::kPrepThreads) {
-      const float v = load_as_f32(P.x, P.xdt, off + k);
+      const float v = load_as_f32(P.x, XDT, off + k);
       m = fmaxf(m, v * v);
     }
   }
@@ -258,6 +259,9 @@ __device__ float prep_block_norms(const BsPrepParams& P, int t, int w0, int nw) 
 }
 
 // One CTA per chunk; see the file comment.
+// TB >= batch: the token loops of the lift compile for TB tokens only, and XDT is the dtype of x:
+// the prep runs once per call from a cold instruction cache, so it carries only the code it runs
+template <int TB, int XDT>
 __global__ void __launch_bounds__(bs::kPrepThreads) gemv_bs_prep_kernel(const BsPrepParams P) {
   // let the dependent GEMV grid launch now: it streams codes at once and waits for this grid
   // before it reads what this grid writes
@@ -292,7 +296,7 @@ __global__ void __launch_bounds__(bs::kPrepThreads) gemv_bs_prep_kernel(const Bs
     const int nblk = span / Bh;
     for (int task = warp; task < P.batch * nblk; task += bs::kPrepWarps) {
       const int tok = task / nblk, b = task - tok * nblk;
-      warp_whiten_block(P.x, P.xdt, (int64_t)tok * P.K, base + b * Bh, E, P.T, P.T.inv_sqrt,
+      warp_whiten_block(P.x, XDT, (int64_t)tok * P.K, base + b * Bh, E, P.T, P.T.inv_sqrt,
                         xs + tok * P.xs_floats + b * Bh);
     }
   } else {
@@ -301,7 +305,7 @@ __global__ void __launch_bounds__(bs::kPrepThreads) gemv_bs_prep_kernel(const Bs
       const int k = base + i;
       float a = 0.f;
       if (k < P.K) {
-        a = load_as_f32(P.x, P.xdt, (int64_t)tok * P.K + k);
+        a = load_as_f32(P.x, XDT, (int64_t)tok * P.K + k);
         if (Bh > 0) {
           if (P.T.chan_scale) a *= __ldg(P.T.chan_scale + k);
           if (P.T.sign && __ldg(P.T.sign + k) < 0) a = -a;
@@ -339,7 +343,7 @@ __global__ void __launch_bounds__(bs::kPrepThreads) gemv_bs_prep_kernel(const Bs
     if (tasks <= bs::kPrepWarps / 2) w0 = tasks;
   }
   for (int tok = 0; tok < P.batch; ++tok) {
-    const float m = bs_warp_max(prep_block_norms(P, tok, w0, bs::kPrepWarps - w0));
+    const float m = bs_warp_max(prep_block_norms<XDT>(P, tok, w0, bs::kPrepWarps - w0));
     if (lane == 0) s_red[tok][warp] = m;
   }
   __syncthreads();
@@ -367,9 +371,9 @@ __global__ void __launch_bounds__(bs::kPrepThreads) gemv_bs_prep_kernel(const Bs
   float Mr[bs::kMaxD];
 #pragma unroll
   for (int i = 0; i < bs::kMaxD; ++i) Mr[i] = (lane_on && i < P.d) ? Ms[i * P.D + jc] : 0.f;
-  float su[bs::kMaxTokens];
+  float su[TB];
 #pragma unroll
-  for (int t = 0; t < bs::kMaxTokens; ++t) su[t] = 0.f;
+  for (int t = 0; t < TB; ++t) su[t] = 0.f;
   if (lane_on) {
     for (int g = gf + warp * gpl + gi; g <= gl; g += bs::kPrepWarps * gpl) {
       const int kg = g * P.d;
@@ -377,7 +381,7 @@ __global__ void __launch_bounds__(bs::kPrepThreads) gemv_bs_prep_kernel(const Bs
       const int e = g * P.D + jc - q0;
       const bool in = e >= 0 && e < qe - q0;
 #pragma unroll
-      for (int tok = 0; tok < bs::kMaxTokens; ++tok) {
+      for (int tok = 0; tok < TB; ++tok) {
         if (tok >= P.batch) continue;
         const float* xt = xs + tok * P.xs_floats + (kg - base);
         float a = 0.f;
@@ -395,7 +399,7 @@ __global__ void __launch_bounds__(bs::kPrepThreads) gemv_bs_prep_kernel(const Bs
   for (int e = (qe - q0) + tid; e < 512; e += bs::kPrepThreads)
     for (int tok = 0; tok < P.batch; ++tok) zc[tok * bs::kZc + e + (e >> 7) * 8] = 0.f;
 #pragma unroll
-  for (int tok = 0; tok < bs::kMaxTokens; ++tok) {
+  for (int tok = 0; tok < TB; ++tok) {
     if (tok < P.batch) {
       const float v = bs_warp_sum(su[tok]);
       if (lane == 0) s_sum[tok][warp] = v;
@@ -817,6 +821,22 @@ BsPlan plan_gemv_bs(int32_t batch, int64_t L, int32_t N, int32_t K, int32_t d, i
   return p;
 }
 
+template <int TB, int XDT>
+static cudaError_t launch_prep_t(const BsPrepParams& Q, const BsPlan& pl, cudaStream_t st) {
+  static int smem_set[64];
+  cudaError_t e = ensure_smem((const void*)gemv_bs_prep_kernel<TB, XDT>, pl.prep_smem, smem_set);
+  if (e != cudaSuccess) return e;
+  gemv_bs_prep_kernel<TB, XDT><<<pl.nchunk, bs::kPrepThreads, pl.prep_smem, st>>>(Q);
+  return cudaGetLastError();
+}
+
+template <int TB>
+static cudaError_t launch_prep(const BsPrepParams& Q, const BsPlan& pl, cudaStream_t st) {
+  if (Q.xdt == LQ_BF16) return launch_prep_t<TB, LQ_BF16>(Q, pl, st);
+  if (Q.xdt == LQ_F16) return launch_prep_t<TB, LQ_F16>(Q, pl, st);
+  return launch_prep_t<TB, LQ_F32>(Q, pl, st);
+}
+
 template <int NT, int HT>
 static cudaError_t launch_bs_nt(const BsPlan& pl, const CUtensorMap& tmap, const BsParams& P,
                                 cudaStream_t st) {
@@ -856,9 +876,6 @@ cudaError_t launch_gemv_bs(const BsPlan& pl, const void* x, int xdt, int32_t bat
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  static int prep_set[64];
-  cudaError_t e = ensure_smem((const void*)gemv_bs_prep_kernel, pl.prep_smem, prep_set);
-  if (e != cudaSuccess) return e;
   BsPrepParams Q{};
   Q.x = x;
   Q.xdt = xdt;
@@ -874,8 +891,10 @@ cudaError_t launch_gemv_bs(const BsPlan& pl, const void* x, int xdt, int32_t bat
   Q.frags = ws.frags;
   Q.csum = ws.csum;
   Q.stok = ws.stok;
-  gemv_bs_prep_kernel<<<pl.nchunk, bs::kPrepThreads, pl.prep_smem, st>>>(Q);
-  e = cudaGetLastError();
+  cudaError_t e = batch <= 1 ? launch_prep<1>(Q, pl, st)
+                  : batch <= 2 ? launch_prep<2>(Q, pl, st)
+                  : batch <= 4 ? launch_prep<4>(Q, pl, st)
+                               : launch_prep<bs::kMaxTokens>(Q, pl, st);
   if (e != cudaSuccess) return e;
 
   BsParams P{};
