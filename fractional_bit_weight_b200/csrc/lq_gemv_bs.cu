@@ -209,6 +209,33 @@ __device__ __forceinline__ float scale_from_bound(float cm, float a2) {
 // of the i-th of them takes the 8 inputs from 8 (32 i + l) + 256 nw r in round r (the loads of
 // four rounds in flight together) and the Bh / 8 lanes of one block add their sums by
 // shuffles. The caller reduces over the CTA.
+// prep_block_norms for Hadamard blocks of fewer than 8 inputs (and the identity: the largest
+// x^2), one block per thread; out of line, as the prep's usual path does not take it
+template <int XDT>
+__device__ __noinline__ float prep_norms_small(const void* x, int K, const Whiten T, int64_t off) {
+  const int tid = threadIdx.x;
+  const int Bh = T.block;
+  float m = 0.f;
+  if (Bh > 0) {
+    for (int b = tid; b < K / Bh; b += bs::kPrepThreads) {
+      float a = 0.f;
+      for (int i = 0; i < Bh; ++i) {
+        const int k = b * Bh + i;
+        float v = load_as_f32(x, XDT, off + k);
+        if (T.chan_scale) v *= __ldg(T.chan_scale + k);
+        a = fmaf(v, v, a);
+      }
+      m = fmaxf(m, a);
+    }
+  } else {
+    for (int k = tid; k < K; k += bs::kPrepThreads) {
+      const float v = load_as_f32(x, XDT, off + k);
+      m = fmaxf(m, v * v);
+    }
+  }
+  return m;
+}
+
 template <int XDT>
 __device__ __forceinline__ float prep_block_norms(const BsPrepParams& P, int t, int w0, int nw) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -238,27 +265,56 @@ __device__ __forceinline__ float prep_block_norms(const BsPrepParams& P, int t, 
       for (int o = 1; o < Bh / 8 && o < 32; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
       if (in) m = fmaxf(m, a);
     }
-  } else if (Bh > 0) {
-    for (int b = tid; b < P.K / Bh; b += bs::kPrepThreads) {
-      float a = 0.f;
-      for (int i = 0; i < Bh; ++i) {
-        const int k = b * Bh + i;
-        float v = load_as_f32(P.x, XDT, off + k);
-        if (P.T.chan_scale) v *= __ldg(P.T.chan_scale + k);
-        a = fmaf(v, v, a);
-      }
-      m = fmaxf(m, a);
-    }
   } else {
-    for (int k = tid; k < P.K; k += bs::kPrepThreads) {
-      const float v = load_as_f32(P.x, XDT, off + k);
-      m = fmaxf(m, v * v);
-    }
+    m = prep_norms_small<XDT>(P.x, P.K, P.T, off);
   }
   return m;
 }
 
 // One CTA per chunk; see the file comment.
+// The whitening of a chunk's inputs for Hadamard blocks of fewer than 32 inputs (and the
+// identity), by the whole CTA through shared memory. Kept out of line: the prep's usual path
+// (blocks of >= 32 inputs, one warp each) then stays compact.
+template <int XDT>
+__device__ __noinline__ void prep_whiten_small(const void* x, int batch, int K, const Whiten T,
+                                               int xs_floats, int base, int span, float* xs) {
+  const int tid = threadIdx.x;
+  const int Bh = T.block;
+  for (int e = tid; e < batch * span; e += bs::kPrepThreads) {
+    const int tok = e / span, i = e - tok * span;
+    const int k = base + i;
+    float a = 0.f;
+    if (k < K) {
+      a = load_as_f32(x, XDT, (int64_t)tok * K + k);
+      if (Bh > 0) {
+        if (T.chan_scale) a *= __ldg(T.chan_scale + k);
+        if (T.sign && __ldg(T.sign + k) < 0) a = -a;
+      }
+    }
+    xs[tok * xs_floats + i] = a;
+  }
+  __syncthreads();
+  if (Bh > 1) {
+    const int half = span / 2;
+    for (int h = 1; h < Bh; h <<= 1) {
+      for (int pp = tid; pp < batch * half; pp += bs::kPrepThreads) {
+        const int tok = pp / half, pi = pp - tok * half;
+        const int lo = pi & (h - 1);
+        const int i = ((pi - lo) << 1) | lo;
+        float* xt = xs + tok * xs_floats;
+        const float a = xt[i], c2 = xt[i + h];
+        xt[i] = a + c2;
+        xt[i + h] = a - c2;
+      }
+      __syncthreads();
+    }
+    for (int e = tid; e < batch * span; e += bs::kPrepThreads) {
+      const int tok = e / span;
+      xs[tok * xs_floats + (e - tok * span)] *= T.inv_sqrt;
+    }
+  }
+}
+
 // TB >= batch: the token loops of the lift compile for TB tokens only, and XDT is the dtype of x:
 // the prep runs once per call from a cold instruction cache, so it carries only the code it runs
 template <int TB, int XDT>
@@ -300,39 +356,7 @@ __global__ void __launch_bounds__(bs::kPrepThreads) gemv_bs_prep_kernel(const Bs
                         xs + tok * P.xs_floats + b * Bh);
     }
   } else {
-    for (int e = tid; e < P.batch * span; e += bs::kPrepThreads) {
-      const int tok = e / span, i = e - tok * span;
-      const int k = base + i;
-      float a = 0.f;
-      if (k < P.K) {
-        a = load_as_f32(P.x, XDT, (int64_t)tok * P.K + k);
-        if (Bh > 0) {
-          if (P.T.chan_scale) a *= __ldg(P.T.chan_scale + k);
-          if (P.T.sign && __ldg(P.T.sign + k) < 0) a = -a;
-        }
-      }
-      xs[tok * P.xs_floats + i] = a;
-    }
-    __syncthreads();
-    if (Bh > 1) {
-      const int half = span / 2;
-      for (int h = 1; h < Bh; h <<= 1) {
-        for (int pp = tid; pp < P.batch * half; pp += bs::kPrepThreads) {
-          const int tok = pp / half, pi = pp - tok * half;
-          const int lo = pi & (h - 1);
-          const int i = ((pi - lo) << 1) | lo;
-          float* xt = xs + tok * P.xs_floats;
-          const float a = xt[i], c2 = xt[i + h];
-          xt[i] = a + c2;
-          xt[i + h] = a - c2;
-        }
-        __syncthreads();
-      }
-      for (int e = tid; e < P.batch * span; e += bs::kPrepThreads) {
-        const int tok = e / span;
-        xs[tok * P.xs_floats + (e - tok * span)] *= P.T.inv_sqrt;
-      }
-    }
+    prep_whiten_small<XDT>(P.x, P.batch, P.K, P.T, P.xs_floats, base, span, xs);
   }
   // 2. every token's largest squared block norm over all of K, by the warps that whitened
   // nothing when that leaves at least half of them (their loads then go out with the
