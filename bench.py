@@ -275,7 +275,7 @@ def _x_tensor(layer):
 
 def kernels_per_step(wl):
     """Kernels one lq_gemm call launches for this workload: as the library reports it, or on a
-    forced route its fixed count (bulk GEMV 1; int8 GEMV and lifted GEMM 2; W, xt, GEMM 3)."""
+    forced route its fixed count (staged GEMV, int8 GEMV and lifted GEMM 2; W, xt, GEMM 3)."""
     fixed = {lq.ROUTE_GEMV_BULK: 2, lq.ROUTE_GEMV_I8: 2, lq.ROUTE_GEMM_TC: 2, lq.ROUTE_GEMM_DQ: 3}
     if wl.route in fixed:
         return fixed[wl.route]
