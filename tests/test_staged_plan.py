@@ -107,3 +107,16 @@ def test_staged_plan_rejects_bad_arguments():
         lq.gemv_staged_plan(1, 8192, 0, 10, 24, 256)
     # a Hadamard block past what the prep holds has no staged plan, without an error
     assert lq.gemv_staged_plan(1, 8192, 8192, 10, 24, 512)["ok"] == 0
+
+
+def test_staged_plan_row_limit_keeps_int32_sums_exact():
+    # The contraction sums, per digit plane, eight products per code byte in int32: the raw byte
+    # unsigned (<= 255) and signed (|.| <= 128), and bit q alone (2^q, q = 1..6), each times a B
+    # digit of magnitude <= 127. The plan takes rows of up to 2^17 lifted coordinates, which must
+    # keep the whole row's sum below 2^31.
+    per_byte = 127 * (255 + 128 + sum(2 ** q for q in range(1, 7)))
+    assert per_byte * (2 ** 17 // 8) < 2 ** 31
+    # d = 1, D = 2 lifts K inputs to 2K coordinates: K = 65536 is the longest row the plan takes
+    assert lq.lifted_bits(65536, 1, 2) == 2 ** 17
+    assert lq.gemv_staged_plan(1, 65536, 4096, 1, 2, 256)["ok"] == 1
+    assert lq.gemv_staged_plan(1, 65536 + 256, 4096, 1, 2, 256)["ok"] == 0
