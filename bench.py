@@ -85,9 +85,14 @@ def dist_setup():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if ws > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=120)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            torch.distributed.init_process_group("nccl", timeout=timeout,
+                                                 device_id=torch.device("cuda", local))
+        else:
+            # a host without GPUs runs only the reference arm (the oracle); its ranks meet over gloo
+            torch.distributed.init_process_group("gloo", timeout=timeout)
     return ws, rank, local
 
 
@@ -99,7 +104,8 @@ def barrier(ws):
 def max_over_ranks(v, ws):
     if ws == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
